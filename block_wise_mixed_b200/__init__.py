@@ -1,0 +1,10 @@
+"""block_wise_mixed_b200 -- block-wise mixed-precision weight-only quantized
+linear layer (64x128 blocks, per-block bits in {0,1,2,3,4,5,6,8}, RTN-g128,
+fp16 scale/zero, bi-directional channel reordering) on NVIDIA B200.
+
+The computation lives in the C-ABI library ``libmpq.so`` (include/mpq.h); this
+package only marshals arguments to it.  ``synth`` draws seeded workloads.
+"""
+from ._lib import (MpqError, PackedLayer, check, linear, linear_host,  # noqa: F401
+                   linear_host_workspace_size, linear_timed, linear_workspace_size, pack,
+                   plan)

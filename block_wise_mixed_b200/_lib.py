@@ -1,0 +1,235 @@
+"""ctypes binding of libmpq.so (C ABI in include/mpq.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch supplies device memory and the current stream.  There is no
+fallback: if libmpq.so is missing the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import numpy as np
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmpq.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "mpq.h")
+
+STATUS = {0: "MPQ_OK", 1: "MPQ_ERR_ARG", 2: "MPQ_ERR_SHAPE", 3: "MPQ_ERR_BITS",
+          4: "MPQ_ERR_PERM", 5: "MPQ_ERR_NONFINITE", 6: "MPQ_ERR_RANGE",
+          7: "MPQ_ERR_WORKSPACE", 8: "MPQ_ERR_CUDA", 9: "MPQ_ERR_TIMEOUT"}
+
+
+class MpqError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        super().__init__("%s%s" % (STATUS.get(status, status), (" in " + where) if where else ""))
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+
+
+class Block(ctypes.Structure):
+    _fields_ = [("code_off", ctypes.c_uint32), ("sz_off", ctypes.c_uint32),
+                ("bits", ctypes.c_uint32), ("bit_prefix", ctypes.c_uint32)]
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("NB", ctypes.c_int32),
+                ("KB", ctypes.c_int32), ("n_units", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("codes_bytes", ctypes.c_uint64),
+                ("n_sz", ctypes.c_uint64), ("bit_total", ctypes.c_uint64),
+                ("seg_off", ctypes.c_uint64 * 9), ("seg_bytes", ctypes.c_uint64 * 9)]
+
+
+class Layer(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("n_units", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("codes", ctypes.c_void_p),
+                ("table", ctypes.c_void_p), ("sched", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+                ("row_perm", ctypes.c_void_p), ("col_perm", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/mpq.h."""
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return re.findall(r"\b(mpq_[a-z_]+)\s*\(", txt)
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libmpq.so not found at %s: build it with "
+                               "block_wise_mixed_b200.build.build()" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        L.mpq_plan.argtypes = [i32, i32, P, ctypes.POINTER(Layout)]
+        L.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
+        L.mpq_pack_workspace_size.restype = sz
+        L.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
+        L.mpq_linear_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
+        L.mpq_linear_workspace_size.restype = sz
+        L.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
+        L.mpq_linear_timed.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P, P, P]
+        L.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
+        L.mpq_linear_host_workspace_size.restype = sz
+        L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
+        L.mpq_check.argtypes = [P, P]
+        L.mpq_status_string.argtypes = [ctypes.c_int]
+        L.mpq_status_string.restype = ctypes.c_char_p
+        for f in ("mpq_plan", "mpq_pack", "mpq_linear", "mpq_linear_timed", "mpq_linear_host",
+                  "mpq_check"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _np_ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _t_ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _raise(st, where):
+    if st != 0:
+        raise MpqError(st, where)
+
+
+def plan(N: int, K: int, bits: np.ndarray) -> Layout:
+    """mpq_plan: layout of a packed layer (host only)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint8).reshape(-1)
+    L = Layout()
+    _raise(lib().mpq_plan(N, K, _np_ptr(bits), ctypes.byref(L)), "mpq_plan")
+    return L
+
+
+@dataclass
+class PackedLayer:
+    """A packed layer in device memory (torch tensors) plus its C view."""
+    layout: Layout
+    codes: object
+    table: object
+    sched: object
+    scales: object
+    zeros: object
+    row_perm: object
+    col_perm: object
+    c: Layer
+
+    @property
+    def N(self):
+        return self.layout.N
+
+    @property
+    def K(self):
+        return self.layout.K
+
+
+def alloc_layer(L: Layout, device, has_row_perm: bool, has_col_perm: bool) -> PackedLayer:
+    import torch
+    u8 = torch.uint8
+
+    def buf(n, dtype=u8):
+        return torch.empty(max(int(n), 1), dtype=dtype, device=device)
+
+    T = L.NB * L.KB
+    codes = buf(L.codes_bytes)
+    table = buf(T * 16)
+    sched = buf((L.n_units + 1) * 4)
+    scales = buf(2 * L.n_sz)
+    zeros = buf(2 * L.n_sz)
+    rp = torch.empty(L.N, dtype=torch.int32, device=device) if has_row_perm else None
+    cp = torch.empty(L.K, dtype=torch.int32, device=device) if has_col_perm else None
+    c = Layer(L.N, L.K, L.n_units, 0, codes.data_ptr(), table.data_ptr(), sched.data_ptr(),
+              scales.data_ptr(), zeros.data_ptr(),
+              rp.data_ptr() if rp is not None else None,
+              cp.data_ptr() if cp is not None else None)
+    return PackedLayer(L, codes, table, sched, scales, zeros, rp, cp, c)
+
+
+def pack(W, bits: np.ndarray, row_perm=None, col_perm=None, ws=None, check=True,
+         stream=None) -> PackedLayer:
+    """mpq_pack.  W: torch bf16 (or int16/uint16 bit patterns) N x K on cuda."""
+    import torch
+    N, K = W.shape
+    bits = np.ascontiguousarray(bits, dtype=np.uint8).reshape(-1)
+    rp = None if row_perm is None else np.ascontiguousarray(row_perm, dtype=np.int32)
+    cp = None if col_perm is None else np.ascontiguousarray(col_perm, dtype=np.int32)
+    L = plan(N, K, bits)
+    P = alloc_layer(L, W.device, rp is not None, cp is not None)
+    if ws is None:
+        ws = torch.empty(lib().mpq_pack_workspace_size(ctypes.byref(L)), dtype=torch.uint8,
+                         device=W.device)
+    Wc = W.contiguous()
+    st = lib().mpq_pack(ctypes.byref(L), Wc.data_ptr(), _np_ptr(bits), _np_ptr(rp), _np_ptr(cp),
+                        ctypes.byref(P.c), ws.data_ptr(), ws.numel(), _stream(stream))
+    _raise(st, "mpq_pack")
+    if check:
+        _raise(lib().mpq_check(ws.data_ptr(), _stream(stream)), "mpq_pack (device)")
+    return P
+
+
+def linear_workspace_size(layer: PackedLayer, M: int) -> int:
+    return lib().mpq_linear_workspace_size(ctypes.byref(layer.c), M)
+
+
+def linear(layer: PackedLayer, x, out=None, ws=None, stream=None):
+    """mpq_linear: y (fp32, M x N) = x (bf16, M x K, cuda) * dequant(W)^T."""
+    import torch
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, layer.N), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(linear_workspace_size(layer, M), 256), dtype=torch.uint8,
+                         device=x.device)
+    st = lib().mpq_linear(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(),
+                          ws.data_ptr(), ws.numel(), _stream(stream))
+    _raise(st, "mpq_linear")
+    return out
+
+
+def linear_timed(layer: PackedLayer, x, out, ws, ev_begin, ev_end, stream=None):
+    """mpq_linear_timed: as linear(), recording torch.cuda.Event objects around
+    the main GEMM kernel."""
+    M = x.shape[0]
+    st = lib().mpq_linear_timed(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(),
+                                ws.data_ptr(), ws.numel(), _stream(stream),
+                                ctypes.c_void_p(ev_begin.cuda_event), ctypes.c_void_p(ev_end.cuda_event))
+    _raise(st, "mpq_linear_timed")
+    return out
+
+
+def linear_host(layer: PackedLayer, x_host, y_host, ws, stream=None):
+    """mpq_linear_host: host (ideally pinned) x -> host y, enqueued on the stream."""
+    M = x_host.shape[0]
+    st = lib().mpq_linear_host(ctypes.byref(layer.c), x_host.data_ptr(), M, y_host.data_ptr(),
+                               ws.data_ptr(), ws.numel(), _stream(stream))
+    _raise(st, "mpq_linear_host")
+    return y_host
+
+
+def linear_host_workspace_size(layer: PackedLayer, M: int) -> int:
+    return lib().mpq_linear_host_workspace_size(ctypes.byref(layer.c), M)
+
+
+def check(ws, stream=None):
+    """mpq_check: synchronize and raise on a device-side error word."""
+    _raise(lib().mpq_check(ws.data_ptr(), _stream(stream)), "device")
+
+
+def table_numpy(P: PackedLayer) -> np.ndarray:
+    return P.table.cpu().numpy().view(np.uint32).reshape(-1, 4)

@@ -1,0 +1,107 @@
+// k_xprep.cuh -- activation prologue: x'[m][j] = x[m][col_perm[j]].
+//
+// SFMP abstract: row-column reordering costs "a small activation reordering
+// overhead during inference" -- this kernel is that step.  It also converts
+// bf16 -> fp16 for the tensor-core operands.  To keep every bf16 value exact
+// in fp16 (8 significant bits fit in 11) and away from fp16 overflow, token m
+// is scaled by an exact power of two 2^e_m chosen from its largest magnitude
+// (e_m = 14 - floor(log2(amax_m)), so amax*2^e lies in [2^14, 2^15)); the
+// GEMM epilogues multiply by tok_scale[m] = 2^-e_m, which is exact.
+//
+// Layouts written:
+//   XP_DECODE : [KB][M][4][16] half2 -- for block column kb, token m and quad
+//               lane t, register r = 4i+j holds the columns (32t+8i+j,
+//               32t+8i+j+4) of that block column: exactly the B fragment of
+//               mma.m16n8k16 that the decode kernel pairs with its code
+//               extraction order.
+//   XP_ROWMAJOR: [M][K] half, K contiguous (the tensor-core kernel's A/B tile
+//               source).
+// Block 0 also clears the workspace error word and the per-block-row
+// counters of the decode kernel's fix-up.
+#pragma once
+#include "common.cuh"
+
+namespace mpq {
+
+enum XprepLayout { XP_DECODE = 0, XP_ROWMAJOR = 1 };
+
+struct XprepParams {
+    const uint16_t* x;         // bf16 bits, M x K
+    const int32_t* col_perm;   // [K] or null
+    __half* xq;                // output (layout above)
+    float* tok_scale;          // [M] = 2^-e_m
+    uint32_t* counters;        // [n_counters] cleared by block 0 (may be null)
+    int n_counters;
+    uint32_t* err;             // cleared by block 0 (may be null)
+    int M, K;
+};
+
+constexpr int XPREP_THREADS = 256;
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
+    // let the GEMM kernel that follows start its prologue early
+    pdl_launch_dependents();
+    __shared__ float red[XPREP_THREADS / 32];
+    const int m = blockIdx.x, tid = threadIdx.x, K = p.K;
+    if (m == 0) {
+        if (tid == 0 && p.err) *p.err = 0u;
+        for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
+    }
+    const uint16_t* xr = p.x + (size_t)m * K;
+    // 1. amax over the row (order-free, so read it unpermuted, 8 values per load)
+    float amax = 0.f;
+    const uint4* xv = reinterpret_cast<const uint4*>(xr);
+    for (int c = tid; c < K / 8; c += XPREP_THREADS) {
+        uint4 v = xv[c];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            float a = fabsf(__uint_as_float(w[h] << 16));
+            float b = fabsf(__uint_as_float(w[h] & 0xffff0000u));
+            // NaN-propagating max: fmaxf would drop NaN
+            amax = (a > amax || a != a) ? a : amax;
+            amax = (b > amax || b != b) ? b : amax;
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        float o = __shfl_xor_sync(0xffffffffu, amax, off);
+        amax = (o > amax || o != o) ? o : amax;
+    }
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    if (tid == 0) {
+        float a = red[0];
+        for (int i = 1; i < XPREP_THREADS / 32; ++i) a = (red[i] > a || red[i] != red[i]) ? red[i] : a;
+        red[0] = a;
+    }
+    __syncthreads();
+    amax = red[0];
+    int e = 0;
+    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -126), 126);
+    if (tid == 0) p.tok_scale[m] = ldexpf(1.f, -e);
+
+    auto load = [&](int j) -> float {
+        int c = p.col_perm ? p.col_perm[j] : j;
+        return ldexpf(__uint_as_float(((uint32_t)xr[c]) << 16), e);
+    };
+    if (LAYOUT == XP_DECODE) {
+        const int KB = K / 128;
+        __half2* out = reinterpret_cast<__half2*>(p.xq);
+        for (int idx = tid; idx < K / 2; idx += XPREP_THREADS) {
+            const int kb = idx >> 6, rem = idx & 63;
+            const int t = rem >> 4, r = rem & 15, i = r >> 2, j = r & 3;
+            const int col = kb * 128 + 32 * t + 8 * i + j;
+            __half2 v = __halves2half2(__float2half_rn(load(col)), __float2half_rn(load(col + 4)));
+            out[((size_t)kb * p.M + m) * 64 + rem] = v;
+        }
+        (void)KB;
+    } else {
+        __half2* out = reinterpret_cast<__half2*>(p.xq + (size_t)m * K);
+        for (int c2 = tid; c2 < K / 2; c2 += XPREP_THREADS)
+            out[c2] = __halves2half2(__float2half_rn(load(2 * c2)), __float2half_rn(load(2 * c2 + 1)));
+    }
+}
+
+}  // namespace mpq

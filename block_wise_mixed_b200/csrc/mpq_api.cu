@@ -1,0 +1,359 @@
+// mpq_api.cu -- the C ABI of libmpq (declared in include/mpq.h): host-side
+// validation, the plan (segment offsets, block table, decode schedule) and
+// the kernel launches.  The library allocates no device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <vector>
+
+#include "../../include/mpq.h"
+#include "common.cuh"
+#include "k_decode.cuh"
+#include "k_pack.cuh"
+#include "k_xprep.cuh"
+
+using namespace mpq;
+
+namespace {
+
+constexpr int kMaxUnits = 444;          // 3 decode CTAs on each of 148 SMs
+constexpr uint64_t kMinUnitBits = 8;    // >= 8 KiB of codes per decode unit
+constexpr int kMaxDecodeTokens = 8;     // tokens per decode launch
+constexpr int kPackRowsPerCta = 16;
+
+inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+inline bool bits_ok(int b) { return b == 0 || b == 1 || b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8; }
+
+// Layout of the plan for (N, K, bits) -- the same arithmetic as mpq_plan.
+mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
+                     std::vector<mpq_block>* table, std::vector<uint32_t>* sched) {
+    if (N <= 0 || K <= 0 || N % 64 != 0 || K % 128 != 0) return MPQ_ERR_SHAPE;
+    const int NB = N / 64, KB = K / 128;
+    const int64_t T = (int64_t)NB * KB;
+    std::memset(L, 0, sizeof *L);
+    L->N = N; L->K = K; L->NB = NB; L->KB = KB;
+    uint64_t count[9] = {0};
+    for (int64_t t = 0; t < T; ++t) {
+        if (!bits_ok(bits[t])) return MPQ_ERR_BITS;
+        ++count[bits[t]];
+    }
+    static const int order[7] = {1, 2, 3, 4, 5, 6, 8};
+    uint64_t off = 0;
+    for (int b : order) {
+        L->seg_off[b] = off;
+        L->seg_bytes[b] = count[b] * 1024u * (uint64_t)b;
+        off += L->seg_bytes[b];
+    }
+    L->codes_bytes = off;
+    if (off >= (1ull << 32)) return MPQ_ERR_SHAPE;
+    uint64_t nz = 0, total = 0;
+    for (int64_t t = 0; t < T; ++t) total += bits[t], nz += bits[t] != 0;
+    L->n_sz = 64u * nz;
+    L->bit_total = total;
+    int64_t units = (int64_t)((total + kMinUnitBits - 1) / kMinUnitBits);
+    units = std::max<int64_t>(1, std::min<int64_t>(units, std::min<int64_t>(kMaxUnits, T)));
+    L->n_units = (int32_t)units;
+    if (table) {
+        table->assign((size_t)T, mpq_block{0, 0, 0, 0});
+        uint64_t seen[9] = {0}, k = 0, pre = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            const int b = bits[t];
+            mpq_block& e = (*table)[(size_t)t];
+            e.bit_prefix = (uint32_t)pre;
+            if (b) {
+                e.code_off = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
+                e.sz_off = (uint32_t)(64u * k);
+                e.bits = (uint32_t)b;
+                ++seen[b];
+                ++k;
+            }
+            pre += (uint64_t)b;
+        }
+    }
+    if (sched) {
+        // unit u starts at the first block whose bit prefix reaches floor(u*S/P)
+        sched->assign((size_t)units + 1, 0u);
+        std::vector<uint64_t> pre((size_t)T + 1, 0);
+        for (int64_t t = 0; t < T; ++t) pre[(size_t)t + 1] = pre[(size_t)t] + bits[t];
+        for (int64_t u = 1; u < units; ++u) {
+            const uint64_t target = (uint64_t)u * total / (uint64_t)units;
+            auto it = std::lower_bound(pre.begin(), pre.begin() + T, target);
+            (*sched)[(size_t)u] = (uint32_t)(it - pre.begin());
+        }
+        (*sched)[(size_t)units] = (uint32_t)T;
+    }
+    return MPQ_OK;
+}
+
+bool perm_ok(const int32_t* p, int n) {
+    std::vector<char> seen((size_t)n, 0);
+    for (int i = 0; i < n; ++i) {
+        if (p[i] < 0 || p[i] >= n || seen[(size_t)p[i]]) return false;
+        seen[(size_t)p[i]] = 1;
+    }
+    return true;
+}
+
+inline mpq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MPQ_OK : MPQ_ERR_CUDA; }
+
+// Workspace carve-up of mpq_linear.
+struct LinearWs {
+    uint32_t* err;
+    uint32_t* counters;
+    float* tok_scale;
+    __half* xq;
+    float* partial;
+    size_t bytes;
+};
+
+LinearWs carve_linear(void* ws, const mpq_layer* layer, int32_t M) {
+    LinearWs w{};
+    const int NB = layer->N / 64;
+    size_t off = 256;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    w.err = reinterpret_cast<uint32_t*>(base);
+    w.counters = reinterpret_cast<uint32_t*>(base + off);
+    off += round256((size_t)NB * 4);
+    w.tok_scale = reinterpret_cast<float*>(base + off);
+    off += round256((size_t)M * 4);
+    w.xq = reinterpret_cast<__half*>(base + off);
+    off += round256((size_t)M * layer->K * 2);
+    w.partial = reinterpret_cast<float*>(base + off);
+    off += round256((size_t)2 * layer->n_units * 64 * 8 * 4);
+    w.bytes = off;
+    return w;
+}
+
+mpq_status check_layer(const mpq_layer* L) {
+    if (!L) return MPQ_ERR_ARG;
+    if (L->N <= 0 || L->K <= 0 || L->N % 64 || L->K % 128) return MPQ_ERR_SHAPE;
+    if (!L->table || !L->sched || L->n_units <= 0) return MPQ_ERR_ARG;
+    return MPQ_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename F>
+cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+std::atomic<uint64_t> g_decode_attr{0};
+
+}  // namespace
+
+extern "C" {
+
+mpq_status mpq_plan(int32_t N, int32_t K, const uint8_t* bits_host, mpq_layout* out) {
+    if (!out || !bits_host) return MPQ_ERR_ARG;
+    return make_plan(N, K, bits_host, out, nullptr, nullptr);
+}
+
+size_t mpq_pack_workspace_size(const mpq_layout*) { return 256; }
+
+mpq_status mpq_pack(const mpq_layout* L, const void* W_dev, const uint8_t* bits_host,
+                    const int32_t* row_perm_host, const int32_t* col_perm_host,
+                    const mpq_layer* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!L || !W_dev || !bits_host || !out) return MPQ_ERR_ARG;
+    mpq_layout chk;
+    std::vector<mpq_block> table;
+    std::vector<uint32_t> sched;
+    mpq_status st = make_plan(L->N, L->K, bits_host, &chk, &table, &sched);
+    if (st != MPQ_OK) return st;
+    if (chk.codes_bytes != L->codes_bytes || chk.n_sz != L->n_sz || chk.n_units != L->n_units)
+        return MPQ_ERR_ARG;
+    if (out->N != L->N || out->K != L->K || out->n_units != L->n_units) return MPQ_ERR_ARG;
+    if (row_perm_host && !perm_ok(row_perm_host, L->N)) return MPQ_ERR_PERM;
+    if (col_perm_host && !perm_ok(col_perm_host, L->K)) return MPQ_ERR_PERM;
+    if (col_perm_host && L->K > 65536) return MPQ_ERR_SHAPE;
+    if ((row_perm_host != nullptr) != (out->row_perm != nullptr) ||
+        (col_perm_host != nullptr) != (out->col_perm != nullptr))
+        return MPQ_ERR_ARG;
+    if (!out->table || !out->sched || (L->codes_bytes && !out->codes) ||
+        (L->n_sz && (!out->scales || !out->zeros)))
+        return MPQ_ERR_ARG;
+    if (!ws || ws_bytes < mpq_pack_workspace_size(L)) return MPQ_ERR_WORKSPACE;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t T = table.size();
+    cudaError_t e = cudaMemcpyAsync(const_cast<mpq_block*>(out->table), table.data(),
+                                    T * sizeof(mpq_block), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(const_cast<uint32_t*>(out->sched), sched.data(),
+                            sched.size() * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && row_perm_host)
+        e = cudaMemcpyAsync(const_cast<int32_t*>(out->row_perm), row_perm_host,
+                            (size_t)L->N * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && col_perm_host)
+        e = cudaMemcpyAsync(const_cast<int32_t*>(out->col_perm), col_perm_host,
+                            (size_t)L->K * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, 4, s);
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    if (L->bit_total == 0) return MPQ_OK;   // nothing to quantize
+
+    PackParams p{};
+    p.W = static_cast<const uint16_t*>(W_dev);
+    p.table = out->table;
+    p.row_perm = out->row_perm;
+    p.col_perm = out->col_perm;
+    p.codes = static_cast<uint8_t*>(const_cast<void*>(out->codes));
+    p.scales = const_cast<uint16_t*>(out->scales);
+    p.zeros = const_cast<uint16_t*>(out->zeros);
+    p.err = static_cast<uint32_t*>(ws);
+    p.N = L->N;
+    p.K = L->K;
+    p.KB = L->KB;
+    p.rows_per_cta = kPackRowsPerCta;
+    const size_t row_bytes = (size_t)L->K * 2;
+    const size_t smem = 2 * row_bytes + ((row_bytes + 15) & ~size_t(15)) + 64;
+    e = cudaFuncSetAttribute(k_pack, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    const int grid = (L->N + kPackRowsPerCta - 1) / kPackRowsPerCta;
+    k_pack<<<grid, PACK_THREADS, smem, s>>>(p);
+    return cuda_status(cudaGetLastError());
+}
+
+size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M) {
+    if (!layer || M < 0) return 0;
+    return carve_linear(nullptr, layer, M).bytes;
+}
+
+mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
+                      void* ws, size_t ws_bytes, void* stream) {
+    return mpq_linear_timed(layer, x_dev, M, y_dev, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
+                            void* ws, size_t ws_bytes, void* stream, void* ev_begin,
+                            void* ev_end) {
+    mpq_status st = check_layer(layer);
+    if (st != MPQ_OK) return st;
+    if (M < 0) return MPQ_ERR_SHAPE;
+    if (M == 0) return MPQ_OK;
+    if (!x_dev || !y_dev) return MPQ_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
+    LinearWs w = carve_linear(ws, layer, M);
+    if (ws_bytes < w.bytes) return MPQ_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int NB = layer->N / 64, KB = layer->K / 128;
+
+    XprepParams xp{};
+    xp.x = static_cast<const uint16_t*>(x_dev);
+    xp.col_perm = layer->col_perm;
+    xp.xq = w.xq;
+    xp.tok_scale = w.tok_scale;
+    xp.counters = w.counters;
+    xp.n_counters = NB;
+    xp.err = w.err;
+    xp.M = M;
+    xp.K = layer->K;
+    k_xprep<XP_DECODE><<<M, XPREP_THREADS, 0, s>>>(xp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+
+    e = ensure_smem_attr(k_decode, (int)sizeof(DecSmem), g_decode_attr);
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    DecodeParams dp{};
+    dp.codes = static_cast<const uint8_t*>(layer->codes);
+    dp.table = layer->table;
+    dp.sched = layer->sched;
+    dp.scales = layer->scales;
+    dp.zeros = layer->zeros;
+    dp.row_perm = layer->row_perm;
+    dp.xq = reinterpret_cast<const uint8_t*>(w.xq);
+    dp.tok_scale = w.tok_scale;
+    dp.y = y_dev;
+    dp.partial = w.partial;
+    dp.counters = w.counters;
+    dp.err = w.err;
+    dp.N = layer->N;
+    dp.K = layer->K;
+    dp.NB = NB;
+    dp.KB = KB;
+    dp.M_total = M;
+    dp.n_units = layer->n_units;
+
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)layer->n_units);
+    cfg.blockDim = dim3(DEC_THREADS);
+    cfg.dynamicSmemBytes = sizeof(DecSmem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (ev_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s) != cudaSuccess)
+        return MPQ_ERR_CUDA;
+    for (int m0 = 0; m0 < M; m0 += kMaxDecodeTokens) {
+        dp.m0 = m0;
+        dp.Mg = std::min(kMaxDecodeTokens, M - m0);
+        e = cudaLaunchKernelEx(&cfg, k_decode, dp);
+        if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    }
+    if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
+        return MPQ_ERR_CUDA;
+    return MPQ_OK;
+}
+
+size_t mpq_linear_host_workspace_size(const mpq_layer* layer, int32_t M) {
+    if (!layer || M < 0) return 0;
+    return mpq_linear_workspace_size(layer, M) + round256((size_t)M * layer->K * 2) +
+           round256((size_t)M * layer->N * 4);
+}
+
+mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host, int32_t M, float* y_host,
+                           void* ws, size_t ws_bytes, void* stream) {
+    mpq_status st = check_layer(layer);
+    if (st != MPQ_OK) return st;
+    if (M < 0) return MPQ_ERR_SHAPE;
+    if (M == 0) return MPQ_OK;
+    if (!x_host || !y_host) return MPQ_ERR_ARG;
+    if (!ws || ws_bytes < mpq_linear_host_workspace_size(layer, M)) return MPQ_ERR_WORKSPACE;
+    const size_t inner = mpq_linear_workspace_size(layer, M);
+    uint8_t* xb = static_cast<uint8_t*>(ws) + inner;
+    float* yb = reinterpret_cast<float*>(xb + round256((size_t)M * layer->K * 2));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(xb, x_host, (size_t)M * layer->K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return MPQ_ERR_CUDA;
+    st = mpq_linear(layer, xb, M, yb, ws, inner, stream);
+    if (st != MPQ_OK) return st;
+    if (cudaMemcpyAsync(y_host, yb, (size_t)M * layer->N * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MPQ_ERR_CUDA;
+    return MPQ_OK;
+}
+
+mpq_status mpq_check(const void* ws, void* stream) {
+    if (!ws) return MPQ_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t err = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MPQ_ERR_CUDA;
+    if (cudaMemcpy(&err, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MPQ_ERR_CUDA;
+    return static_cast<mpq_status>(err);
+}
+
+const char* mpq_status_string(mpq_status s) {
+    switch (s) {
+        case MPQ_OK: return "MPQ_OK";
+        case MPQ_ERR_ARG: return "MPQ_ERR_ARG";
+        case MPQ_ERR_SHAPE: return "MPQ_ERR_SHAPE";
+        case MPQ_ERR_BITS: return "MPQ_ERR_BITS";
+        case MPQ_ERR_PERM: return "MPQ_ERR_PERM";
+        case MPQ_ERR_NONFINITE: return "MPQ_ERR_NONFINITE";
+        case MPQ_ERR_RANGE: return "MPQ_ERR_RANGE";
+        case MPQ_ERR_WORKSPACE: return "MPQ_ERR_WORKSPACE";
+        case MPQ_ERR_CUDA: return "MPQ_ERR_CUDA";
+        case MPQ_ERR_TIMEOUT: return "MPQ_ERR_TIMEOUT";
+    }
+    return "MPQ_ERR_UNKNOWN";
+}
+
+}  // extern "C"

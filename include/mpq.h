@@ -1,0 +1,197 @@
+/*
+ * mpq.h -- C ABI of the block-wise mixed-precision weight-only quantized
+ * linear layer for NVIDIA B200 (sm_100a).
+ *
+ *   y = x * dequant(W)^T
+ *
+ * Method (web pages on the subject, cited by title and section):
+ *   "ScaleBITS: Scalable Bitwidth Search for Hardware-Aligned Mixed-Precision
+ *   LLMs" -- abstract and summary page, section "Approach": the weight matrix
+ *   is partitioned into hardware-aligned 64x128 blocks, each with its own bit
+ *   width under a global budget, after rows and columns are reordered so that
+ *   sensitive weights cluster; "Key results"/"Limitations": the scalar
+ *   quantizer is round-to-nearest with group size 128; "Surprising findings":
+ *   0- or 1-bit minimum precision.
+ *   "SFMP: Fine-Grained, Hardware-Friendly and Search-Free Mixed-Precision
+ *   Quantization for Large Language Models" -- abstract: block-wise mixed
+ *   precision with row-column reordering and a small activation reordering
+ *   step at inference.
+ *   "TileQuant: Tile as the Precision-Allocation Unit for LLM Mixed-Precision
+ *   Post-Training Quantization" -- abstract: the precision map guides compact
+ *   weight buffers that the kernel streams.
+ *
+ * Definitions (the pages give no formulas; these readings are the library's):
+ *   W is N x K (out x in, nn.Linear layout), bf16, row-major.  With
+ *   permutations P_r (N) and P_c (K), W'[i][j] = W[P_r[i]][P_c[j]].
+ *   Block (nb, kb) of W' is rows 64nb..64nb+63, columns 128kb..128kb+127;
+ *   block id t = nb*KB + kb; each block has bits[t] in {0,1,2,3,4,5,6,8}.
+ *   Each block row is one RTN group of 128 weights:
+ *     lo = min(min w, 0), hi = max(max w, 0), d = hi - lo, qmax = 2^b - 1,
+ *     s  = smallest fp16 h with h*qmax >= d  (s = 1 if d == 0),
+ *     z  = rne(-lo / s) (an integer in [0, qmax], stored as fp16),
+ *     q  = clamp(rne(w / s) + z, 0, qmax),   w_hat = (q - z) * s.
+ *   A 0-bit block has no codes and dequantizes to zero.
+ *   y[m][P_r[i]] = sum_j x[m][P_c[j]] * w_hat'[i][j]   (y is fp32).
+ *
+ * Packed format v1 (the library's own; the pages name no layout):
+ *   codes   -- segments for b = 1,2,3,4,5,6,8 in that order, each holding the
+ *              payloads of all b-bit blocks in ascending t.  A payload is
+ *              1024*b bytes: the code's "pieces" (1->[1], 2->[2], 3->[2,1],
+ *              4->[4], 5->[4,1], 6->[4,2], 8->[8]; q = lo | hi << width(lo)),
+ *              low piece first; a p-bit piece is 64 rows x 16p bytes,
+ *              row-major; in a row, code j sits in little-endian 32-bit word
+ *              j/(32/p) at bit (j%(32/p))*p.
+ *   scales, zeros -- fp16 bit patterns, 64 per non-zero block, in ascending t;
+ *              row r of block t is at table[t].sz_off + r.
+ *   table   -- one mpq_block per block (ascending t).
+ *   sched   -- n_units+1 block ids: decode work unit u covers blocks
+ *              [sched[u], sched[u+1]) in row-major order, cut so that every
+ *              unit holds about the same number of code bytes.
+ *
+ * Conventions:
+ *   - The caller owns every buffer.  The library allocates no device memory
+ *     and keeps no global state; calls are asynchronous on `stream` (a
+ *     cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - Errors that the host can see are returned at once and nothing is
+ *     launched.  Errors found in device data (non-finite W, a group with no
+ *     representable scale) or a device wait that ran out are written to an
+ *     error word at the start of the workspace; mpq_check() reports them.
+ *   - A launch failure returns MPQ_ERR_CUDA.
+ *   - Limits: N % 64 == 0, K % 128 == 0, N, K > 0, K <= 65536 when a column
+ *     permutation is given, codes_bytes < 2^32; M >= 0 (M == 0 is a no-op).
+ */
+#ifndef MPQ_H
+#define MPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MPQ_OK = 0,
+    MPQ_ERR_ARG = 1,        /* NULL pointer or inconsistent argument        */
+    MPQ_ERR_SHAPE = 2,      /* N % 64, K % 128, N or K <= 0, M < 0, too big  */
+    MPQ_ERR_BITS = 3,       /* a bit width outside {0,1,2,3,4,5,6,8}         */
+    MPQ_ERR_PERM = 4,       /* a permutation that is not a bijection         */
+    MPQ_ERR_NONFINITE = 5,  /* NaN/Inf in W (device-detected)               */
+    MPQ_ERR_RANGE = 6,      /* no fp16 scale, or qmax*s > 65504 (device)    */
+    MPQ_ERR_WORKSPACE = 7,  /* workspace missing or too small               */
+    MPQ_ERR_CUDA = 8,       /* a CUDA call failed                           */
+    MPQ_ERR_TIMEOUT = 9     /* a bounded device wait ran out (device)       */
+} mpq_status;
+
+/* One block of the table (16 bytes). */
+typedef struct {
+    uint32_t code_off;    /* byte offset of the payload in `codes` (0 if 0-bit) */
+    uint32_t sz_off;      /* index of the block's row 0 in scales/zeros          */
+    uint32_t bits;        /* 0,1,2,3,4,5,6 or 8                                  */
+    uint32_t bit_prefix;  /* sum of bits of all blocks with a smaller id        */
+} mpq_block;
+
+/* Sizes of a packed layer; filled by mpq_plan. */
+typedef struct {
+    int32_t N, K, NB, KB;    /* NB = N/64, KB = K/128                          */
+    int32_t n_units;         /* decode work units (sched has n_units+1 entries) */
+    int32_t reserved;
+    uint64_t codes_bytes;    /* = 1024 * bit_total                              */
+    uint64_t n_sz;           /* = 64 * number of non-zero blocks                */
+    uint64_t bit_total;      /* sum of the per-block bits                       */
+    uint64_t seg_off[9];     /* byte offset of segment b (index = bit width)    */
+    uint64_t seg_bytes[9];   /* bytes of segment b ([0] and [7] are 0)          */
+} mpq_layout;
+
+/* A packed layer: device pointers to caller-owned buffers of the sizes in
+ * mpq_layout.  mpq_pack writes these buffers; mpq_linear reads them. */
+typedef struct {
+    int32_t N, K;
+    int32_t n_units;
+    int32_t reserved;
+    const void* codes;           /* uint8  [codes_bytes]                        */
+    const mpq_block* table;      /* [NB*KB]                                      */
+    const uint32_t* sched;       /* [n_units + 1]                                */
+    const uint16_t* scales;      /* fp16 bits [n_sz]                             */
+    const uint16_t* zeros;       /* fp16 bits [n_sz]                             */
+    const int32_t* row_perm;     /* int32 [N]; NULL = identity                   */
+    const int32_t* col_perm;     /* int32 [K]; NULL = identity                   */
+} mpq_layer;
+
+/* Host only.  Validates N, K and the bit map (uint8, NB*KB, block id order)
+ * and fills `out`: segment offsets/sizes, codes_bytes, n_sz, bit_total and
+ * the number of decode work units.  Block partition: ScaleBITS summary,
+ * "Approach"; bit set and budget: ScaleBITS abstract, "Key results".
+ * Errors: MPQ_ERR_ARG, MPQ_ERR_SHAPE, MPQ_ERR_BITS. */
+mpq_status mpq_plan(int32_t N, int32_t K, const uint8_t* bits_host,
+                    mpq_layout* out);
+
+/* Workspace bytes that mpq_pack needs (the error word). */
+size_t mpq_pack_workspace_size(const mpq_layout* L);
+
+/* Quantize and pack W (ScaleBITS summary "Approach" + "Key results": RTN-g128
+ * per 64x128 block after reordering; TileQuant abstract: compact buffers).
+ *   L              layout from mpq_plan for the same N, K and bits.
+ *   W_dev          bf16 bit patterns, N x K row-major, ORIGINAL order, device.
+ *   bits_host      uint8 [NB*KB] (host).
+ *   row_perm_host, col_perm_host   int32 permutations (host) or NULL.
+ *   out            buffers to fill (device): codes, table, sched, scales,
+ *                  zeros; out->row_perm / col_perm receive copies of the host
+ *                  permutations and must be NULL exactly when those are NULL.
+ *   ws, ws_bytes   device workspace (>= mpq_pack_workspace_size).
+ * The result is a pure function of the inputs (byte-deterministic).
+ * Host errors: ARG, SHAPE, BITS, PERM, WORKSPACE; device errors (mpq_check):
+ * NONFINITE, RANGE.  Outputs are unspecified after a device error. */
+mpq_status mpq_pack(const mpq_layout* L, const void* W_dev,
+                    const uint8_t* bits_host, const int32_t* row_perm_host,
+                    const int32_t* col_perm_host, const mpq_layer* out,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes that mpq_linear needs for M tokens. */
+size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
+
+/* y = x * dequant(W)^T for M tokens, including the activation column
+ * reordering x'[m][j] = x[m][P_c[j]] (SFMP abstract: "activation reordering
+ * overhead during inference") and the inverse output reordering
+ * y[m][P_r[i]] = y'[m][i].
+ *   x_dev   bf16 bit patterns, M x K row-major (device).
+ *   y_dev   fp32, M x N row-major, original output order (device).
+ *   ws      device workspace of >= mpq_linear_workspace_size(layer, M) bytes,
+ *           256-byte aligned; its contents need no initialization.
+ * Uses a memory-bound decode kernel for M <= 32 and a tensor-core kernel for
+ * larger M.  Non-finite x gives non-finite y (no error).
+ * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT. */
+mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M,
+                      float* y_dev, void* ws, size_t ws_bytes, void* stream);
+
+/* mpq_linear that also records two CUDA events (cudaEvent_t as void*; either
+ * may be NULL) on `stream`: ev_begin right before the first launch of the
+ * main GEMM kernel and ev_end right after its last launch, so a caller can
+ * time that kernel alone with events (the activation prologue is outside).
+ * Same arguments, results and errors as mpq_linear. */
+mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M,
+                            float* y_dev, void* ws, size_t ws_bytes, void* stream,
+                            void* ev_begin, void* ev_end);
+
+/* The same product with HOST activations and outputs: copies x_host (bf16,
+ * M x K) into the workspace, runs mpq_linear and copies y back to y_host
+ * (fp32, M x N), all on `stream`; returns after enqueueing (synchronize the
+ * stream before reading y_host).  Use pinned host memory for asynchrony.
+ * ws must hold mpq_linear_host_workspace_size(layer, M) bytes. */
+size_t mpq_linear_host_workspace_size(const mpq_layer* layer, int32_t M);
+mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host,
+                           int32_t M, float* y_host, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream` and returns the device error word stored in `ws` by
+ * the last mpq_pack / mpq_linear on that workspace (MPQ_OK if none). */
+mpq_status mpq_check(const void* ws, void* stream);
+
+/* Human-readable name of a status. */
+const char* mpq_status_string(mpq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MPQ_H */

@@ -1,0 +1,111 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/mpq.h declares, and its host-side plan and argument validation
+agree with the oracle.  No compute call is made here."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from block_wise_mixed_b200 import _lib as B
+from block_wise_mixed_b200 import build, synth
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return B.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = B.header_functions()
+    assert {"mpq_plan", "mpq_pack", "mpq_linear", "mpq_check", "mpq_status_string",
+            "mpq_pack_workspace_size", "mpq_linear_workspace_size", "mpq_linear_host",
+            "mpq_linear_host_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in B.STATUS.items():
+        assert lib.mpq_status_string(code).decode() == name
+
+
+def test_struct_sizes():
+    assert ctypes.sizeof(B.Block) == 16
+    assert ctypes.sizeof(B.Layout) == 4 * 6 + 8 * 3 + 8 * 18
+    assert ctypes.sizeof(B.Layer) == 16 + 7 * 8
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_plan_matches_oracle(lib, oracle, cfg):
+    L = synth.config_layer(cfg, 0)
+    got = B.plan(L.N, L.K, L.bits)
+    ref, _ = oracle.plan(L.N, L.K, L.bits)
+    assert (got.N, got.K, got.NB, got.KB) == (ref.N, ref.K, ref.NB, ref.KB)
+    assert got.codes_bytes == ref.codes_bytes and got.n_sz == ref.n_sz
+    assert got.bit_total == ref.bit_total
+    assert list(got.seg_off) == ref.seg_off and list(got.seg_bytes) == ref.seg_bytes
+    assert 1 <= got.n_units <= 444
+
+
+@pytest.mark.parametrize("N,K,bits,err", [
+    (63, 128, [1], "MPQ_ERR_SHAPE"), (64, 100, [1], "MPQ_ERR_SHAPE"),
+    (0, 128, [1], "MPQ_ERR_SHAPE"), (64, 128, [7], "MPQ_ERR_BITS"),
+    (64, 256, [1, 9], "MPQ_ERR_BITS")])
+def test_plan_errors(lib, N, K, bits, err):
+    with pytest.raises(B.MpqError) as ei:
+        B.plan(N, K, np.array(bits, np.uint8))
+    assert ei.value.name == err
+
+
+def _fake_layer(L, rp=False, cp=False):
+    # non-null placeholders: these calls must fail validation before any
+    # device access, so the pointers are never dereferenced
+    return B.Layer(L.N, L.K, L.n_units, 0, 16, 16, 16, 16, 16, 16 if rp else None,
+                   16 if cp else None)
+
+
+def test_pack_host_validation(lib):
+    N, K = 128, 256
+    bits = np.array([1, 2, 3, 4], np.uint8)
+    L = B.plan(N, K, bits)
+    out = _fake_layer(L, rp=True, cp=True)
+    rp = np.arange(N, dtype=np.int32)
+    cp = np.arange(K, dtype=np.int32)
+    bad = rp.copy()
+    bad[3] = bad[4]
+    P = ctypes.c_void_p
+
+    def call(bits_=bits, rp_=rp, cp_=cp, out_=out, ws=256, L_=L):
+        return lib.mpq_pack(ctypes.byref(L_), P(16), bits_.ctypes.data,
+                            None if rp_ is None else rp_.ctypes.data,
+                            None if cp_ is None else cp_.ctypes.data,
+                            ctypes.byref(out_), P(256 if ws else 0), ws, None)
+    assert B.STATUS[call(rp_=bad)] == "MPQ_ERR_PERM"
+    bad_c = cp.copy()
+    bad_c[0] = K
+    assert B.STATUS[call(cp_=bad_c)] == "MPQ_ERR_PERM"
+    assert B.STATUS[call(bits_=np.array([1, 2, 7, 4], np.uint8))] == "MPQ_ERR_BITS"
+    # a permutation given on the host needs a device buffer for its copy
+    assert B.STATUS[call(out_=_fake_layer(L))] == "MPQ_ERR_ARG"
+    assert B.STATUS[call(ws=0)] == "MPQ_ERR_WORKSPACE"
+    assert B.STATUS[call(ws=16)] == "MPQ_ERR_WORKSPACE"
+    # layout that does not belong to these bits
+    L2 = B.plan(N, K, np.array([2, 2, 3, 4], np.uint8))
+    assert B.STATUS[call(L_=L2)] == "MPQ_ERR_ARG"
+
+
+def test_linear_host_validation(lib):
+    L = B.plan(128, 256, np.array([1, 2, 3, 4], np.uint8))
+    layer = _fake_layer(L)
+    P = ctypes.c_void_p
+    need = lib.mpq_linear_workspace_size(ctypes.byref(layer), 4)
+    assert need > 0
+    # M == 0 is an empty batch: nothing to do
+    assert lib.mpq_linear(ctypes.byref(layer), P(16), 0, P(16), P(256), need, None) == 0
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), P(16), -1, P(16), P(256), need, None)] == "MPQ_ERR_SHAPE"
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), P(16), 4, P(16), P(256), need - 1, None)] == "MPQ_ERR_WORKSPACE"
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), P(16), 4, P(16), P(8), need, None)] == "MPQ_ERR_WORKSPACE"
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), None, 4, P(16), P(256), need, None)] == "MPQ_ERR_ARG"
+    bad = B.Layer(100, 256, L.n_units, 0, 16, 16, 16, 16, 16, None, None)
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(bad), P(16), 4, P(16), P(256), need, None)] == "MPQ_ERR_SHAPE"

@@ -1,0 +1,234 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Bars: packed codes, table, scales and zeros bit-exact; y within
+|y - y_ref| <= 1e-3 * sum_k |x_k * w_hat_k| per output and relative Frobenius
+error <= 5e-4 (y is fp32).  Inputs are seeded synthetic layers with the
+pages' Llama-2/3 shapes (see block_wise_mixed_b200/synth.py).
+"""
+import numpy as np
+import pytest
+
+from block_wise_mixed_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+PER_OUT = 1e-3
+FROB = 5e-4
+
+
+@pytest.fixture(scope="module")
+def mpq():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_wise_mixed_b200 import build
+    build.build()
+    import block_wise_mixed_b200 as m
+    return m
+
+
+def dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def pack_gpu(mpq, L):
+    return mpq.pack(dev(L.W), L.bits, L.row_perm, L.col_perm)
+
+
+def assert_pack_equal(P, R):
+    import torch
+    torch.cuda.synchronize()
+    T = R.table.shape[0]
+    got_table = P.table.cpu().numpy().view(np.uint32).reshape(-1, 4)[:T]
+    assert np.array_equal(got_table, R.table)
+    assert np.array_equal(P.codes.cpu().numpy()[:R.codes.size], R.codes)
+    assert np.array_equal(P.scales.cpu().numpy().view(np.uint16)[:R.scales.size], R.scales)
+    assert np.array_equal(P.zeros.cpu().numpy().view(np.uint16)[:R.zeros.size], R.zeros)
+
+
+def check_sched(P, bits):
+    sched = P.sched.cpu().numpy().view(np.uint32)[:P.layout.n_units + 1].astype(np.int64)
+    T = len(bits)
+    assert sched[0] == 0 and sched[-1] == T
+    assert np.all(np.diff(sched) >= 0)
+    pre = np.concatenate([[0], np.cumsum(bits.astype(np.int64))])
+    S, U = pre[-1], len(sched) - 1
+    for u in range(1, U):   # unit u begins at the first block reaching floor(u*S/U) bits
+        tgt = u * S // U
+        assert pre[sched[u]] >= tgt and (sched[u] == 0 or pre[sched[u] - 1] < tgt)
+
+
+def assert_y_close(y, y_ref, bnd):
+    err = np.abs(y.astype(np.float64) - y_ref)
+    bad = err > PER_OUT * bnd
+    assert not bad.any(), "per-output bound violated at %d outputs, worst ratio %g" % (
+        bad.sum(), float(np.max(err / np.maximum(bnd, 1e-300))))
+    nrm = np.linalg.norm(y_ref)
+    if nrm > 0:
+        assert np.linalg.norm(y - y_ref) / nrm <= FROB
+    else:
+        assert np.all(y == 0)
+
+
+def run_linear(mpq, P, x_bits):
+    import torch
+    y = mpq.linear(P, dev(x_bits))
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_pack_bit_exact_configs(mpq, oracle, cfg):
+    L = synth.config_layer(cfg, 0)
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    check_sched(P, L.bits)
+
+
+@pytest.mark.parametrize("cfg,M", [(1, 1), (1, 2), (1, 3), (1, 7), (1, 8), (1, 9), (1, 17),
+                                   (1, 33), (2, 1), (2, 4), (2, 8)])
+def test_linear_configs(mpq, oracle, cfg, M):
+    L = synth.config_layer(cfg, 0)
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    x = synth.make_x(synth.seed_of(cfg, 0), M, L.K)
+    y_ref, bnd = oracle.linear(R, x)
+    assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 6, 8])
+def test_single_block_each_width(mpq, oracle, b):
+    L = synth.make_layer("blk", 64, 128, float(b), 900 + b, "random", allowed=(b,))
+    assert np.all(L.bits == b)
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    for M in (1, 5):
+        x = synth.make_x(900 + b, M, L.K)
+        y_ref, bnd = oracle.linear(R, x)
+        assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
+
+
+@pytest.mark.parametrize("kind", ["all0", "all8", "one_nonzero", "identity", "uniform2"])
+def test_edge_layers(mpq, oracle, kind):
+    N, K = 384, 1024
+    L = synth.make_layer("edge", N, K, 2.5, 777, "random")
+    if kind == "all0":
+        L.bits[:] = 0
+    elif kind == "all8":
+        L.bits[:] = 8
+    elif kind == "one_nonzero":
+        L.bits[:] = 0
+        L.bits[len(L.bits) // 3] = 3
+    elif kind == "identity":
+        L.row_perm = None
+        L.col_perm = None
+    elif kind == "uniform2":
+        L.bits[:] = 2
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    check_sched(P, L.bits)
+    for M in (1, 3, 8):
+        x = synth.make_x(777, M, K)
+        y_ref, bnd = oracle.linear(R, x)
+        y = run_linear(mpq, P, x)
+        assert_y_close(y, y_ref, bnd)
+        if kind == "all0":
+            assert np.all(y == 0)
+
+
+def test_zero_rows_and_zero_x(mpq, oracle):
+    """An all-zero activation gives exactly 0; so do rows of W that are zero."""
+    L = synth.make_layer("z", 256, 512, 3.0, 31, "random")
+    W = L.W.copy()
+    W[L.row_perm[:64]] = 0          # one whole block row of W' is zero
+    P = mpq.pack(dev(W), L.bits, L.row_perm, L.col_perm)
+    R = oracle.pack(W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    x = synth.make_x(31, 2, L.K)
+    y = run_linear(mpq, P, x)
+    y_ref, bnd = oracle.linear(R, x)
+    assert_y_close(y, y_ref, bnd)
+    assert np.all(y[:, L.row_perm[:64]] == 0)
+    y0 = run_linear(mpq, P, np.zeros_like(x))
+    assert np.all(y0 == 0)
+
+
+def test_extreme_activation_scale(mpq, oracle):
+    """Per-token power-of-two scaling keeps huge and tiny bf16 tokens exact in fp16."""
+    L = synth.make_layer("s", 128, 256, 4.0, 41, "random")
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    xf = synth.bf16_bits_to_f32(synth.make_x(41, 3, L.K))
+    xf = xf * np.array([[3e4], [1e-30], [1e30]], np.float32)
+    x = synth.f32_to_bf16_bits(xf)
+    y_ref, bnd = oracle.linear(R, x)
+    assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
+
+
+def test_device_errors(mpq):
+    import torch
+    from block_wise_mixed_b200 import MpqError
+    L = synth.make_layer("e", 128, 256, 2.0, 51, "random")
+    W = L.W.copy()
+    W[L.row_perm[5], L.col_perm[7]] = 0x7FC0         # NaN in block (0, 0)
+    bits = np.full_like(L.bits, 2)
+    with pytest.raises(MpqError) as ei:
+        mpq.pack(dev(W), bits, L.row_perm, L.col_perm)
+    assert ei.value.name == "MPQ_ERR_NONFINITE"
+    W = L.W.copy()
+    W[0, 0] = synth.f32_to_bf16_bits(np.array([1e30], np.float32))[0]
+    with pytest.raises(MpqError) as ei:
+        mpq.pack(dev(W), bits)
+    assert ei.value.name == "MPQ_ERR_RANGE"
+    # the context is still usable afterwards
+    P = mpq.pack(dev(L.W), bits)
+    torch.cuda.synchronize()
+
+
+def test_deterministic(mpq):
+    L = synth.config_layer(2, 0)
+    P = pack_gpu(mpq, L)
+    x = dev(synth.make_x(synth.seed_of(2, 0), 4, L.K))
+    y1 = mpq.linear(P, x).cpu().numpy()
+    y2 = mpq.linear(P, x).cpu().numpy()
+    assert np.array_equal(y1, y2)
+
+
+def test_linear_host_entry_point(mpq, oracle):
+    import torch
+    L = synth.config_layer(1, 0)
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    x = synth.make_x(synth.seed_of(1, 0), 3, L.K)
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    yh = torch.empty((3, L.N), dtype=torch.float32).pin_memory()
+    ws = torch.empty(mpq.linear_host_workspace_size(P, 3), dtype=torch.uint8, device="cuda")
+    mpq.linear_host(P, xh, yh, ws)
+    torch.cuda.synchronize()
+    y_ref, bnd = oracle.linear(R, x)
+    assert_y_close(yh.numpy(), y_ref, bnd)
+
+
+# ---------------------------------------------------------------------------
+# Full-size layers in the benchmark's launch configuration, checked on
+# sampled output rows the oracle computes one by one.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("cfg,proj,Ms", [(3, 0, (1, 8, 16, 32)), (3, 2, (1, 8)),
+                                         (4, 1, (1, 4, 16)), (4, 3, (1,))])
+def test_full_size_sampled(mpq, oracle, cfg, proj, Ms):
+    L = synth.config_layer(cfg, proj)
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    check_sched(P, L.bits)
+    rng = np.random.default_rng(cfg * 10 + proj)
+    rows = np.sort(rng.choice(L.N, 96, replace=False)).astype(np.int32)
+    for M in Ms:
+        x = synth.make_x(synth.seed_of(cfg, proj), M, L.K)
+        y = run_linear(mpq, P, x)
+        y_ref, bnd = oracle.linear_rows(R, x, rows)
+        assert_y_close(y[:, rows], y_ref, bnd)
