@@ -198,7 +198,8 @@ def build_replicas(mpq, P, R):
     return reps
 
 
-def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sampler=None):
+def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sampler=None,
+               quick=False):
     """Times `steps` mpq_linear calls over L2-busting replicas of one layer.
     Returns a dict of measurements."""
     import torch
@@ -246,10 +247,17 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     clocks = sampler.stop() if sampler else None
     ms_total = e0.elapsed_time(e1)
     ms_step = reduce_max_over_ranks(ms_total, world, device) / steps
+    nbytes = algorithmic_bytes(L.N, L.K, M, lay.codes_bytes, lay.n_sz, T,
+                               L.row_perm is not None, L.col_perm is not None)
+    if quick:
+        return dict(N=L.N, K=L.K, M=M, bytes=nbytes, ms_step=ms_step, replicas=R)
 
     # main-kernel time alone, events recorded by the library around it
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
+    for a, b in evs:        # torch creates the CUDA events on first record
+        a.record(stream)
+        b.record(stream)
     torch.cuda.synchronize(device)
     for s in range(steps):
         mpq.linear_timed(reps[s % R], x, y, ws, evs[s][0], evs[s][1])
@@ -272,8 +280,6 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     torch.cuda.synchronize(device)
     e2e_ms = reduce_max_over_ranks(h0.elapsed_time(h1), world, device) / steps
 
-    nbytes = algorithmic_bytes(L.N, L.K, M, lay.codes_bytes, lay.n_sz, T,
-                               L.row_perm is not None, L.col_perm is not None)
     kbytes = (lay.codes_bytes + 4 * lay.n_sz + 16 * T + 4 * (L.N if L.row_perm is not None else 0)
               + 2 * M * L.K + 4 * M * L.N)
     out = dict(N=L.N, K=L.K, M=M, avg_bits=float(L.bits.mean()), f0=float((L.bits == 0).mean()),
@@ -310,6 +316,17 @@ def run_gpu(args):
     peaks, peak_src = load_peaks()
     layer = synth.config_layer(HEADLINE_CFG, 0)
     M = 1
+    if args.quick:
+        # the timed loop only (for profiler captures of the same command)
+        r = time_layer(mpq, layer, M, args.steps, args.warmup, world, device, soak_s=0.0,
+                       quick=True)
+        if rank == 0:
+            print(json.dumps({"quick": True, "ms_per_step": r["ms_step"],
+                              "GBps": r["bytes"] / (r["ms_step"] * 1e-3) / 1e9}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     sampler = ClockSampler(local)
     r = time_layer(mpq, layer, M, args.steps, args.warmup, world, device, sampler=sampler)
 
@@ -421,6 +438,8 @@ def main(argv=None):
     ap.add_argument("--extra", action="store_true", help="also time the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="timed loop only, no soak/e2e/CPU baseline (for ncu)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

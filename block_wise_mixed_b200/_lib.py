@@ -144,7 +144,7 @@ def alloc_layer(L: Layout, device, has_row_perm: bool, has_col_perm: bool) -> Pa
     u8 = torch.uint8
 
     def buf(n, dtype=u8):
-        return torch.empty(max(int(n), 1), dtype=dtype, device=device)
+        return torch.empty(max(int(n), 16), dtype=dtype, device=device)
 
     T = L.NB * L.KB
     codes = buf(L.codes_bytes)
@@ -206,6 +206,9 @@ def linear_timed(layer: PackedLayer, x, out, ws, ev_begin, ev_end, stream=None):
     """mpq_linear_timed: as linear(), recording torch.cuda.Event objects around
     the main GEMM kernel."""
     M = x.shape[0]
+    for ev in (ev_begin, ev_end):
+        if ev.cuda_event == 0:   # torch creates the CUDA event on first record
+            ev.record()
     st = lib().mpq_linear_timed(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(),
                                 ws.data_ptr(), ws.numel(), _stream(stream),
                                 ctypes.c_void_p(ev_begin.cuda_event), ctypes.c_void_p(ev_end.cuda_event))
