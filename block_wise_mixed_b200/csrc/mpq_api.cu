@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "../../include/mpq.h"
@@ -338,6 +339,52 @@ mpq_status mpq_check(const void* ws, void* stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return MPQ_ERR_CUDA;
     if (cudaMemcpy(&err, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MPQ_ERR_CUDA;
     return static_cast<mpq_status>(err);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// mpq_linear_noalloc: mpq_linear for callers that cannot allocate device
+// memory.  Its scratch is this fixed array, which every device that loads the
+// library holds until the process exits.  Host code must not hand the
+// array's name to a kernel (in host code it is only a stand-in for the
+// symbol); the device address is looked up once per device with
+// cudaGetSymbolAddress, with that device current, on the first call there.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MPQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+}  // namespace
+
+extern "C" {
+
+mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t M,
+                              float* y_dev, void* stream) {
+    mpq_status st = check_layer(layer);
+    if (st != MPQ_OK) return st;
+    if (M < 0) return MPQ_ERR_SHAPE;
+    if (M == 0) return MPQ_OK;
+    if (mpq_linear_workspace_size(layer, M) > (size_t)MPQ_NOALLOC_SCRATCH_BYTES)
+        return MPQ_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MPQ_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return MPQ_ERR_ARG;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+                return MPQ_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // The existing path clears the scratch's error word and fix-up counters
+    // (the only parts that must start at zero) at the start of every call.
+    return mpq_linear(layer, x_dev, M, y_dev, scratch, (size_t)MPQ_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 const char* mpq_status_string(mpq_status s) {

@@ -183,6 +183,30 @@ mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host,
                            int32_t M, float* y_host, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* mpq_linear for callers that cannot allocate device memory, and so cannot
+ * pass a workspace: e.g. an inference-engine plugin whose device memory is
+ * fixed when it is initialized, or a host program whose allocator is not
+ * reachable through this C ABI.  (The paper has no counterpart: this is a
+ * deployment convenience of the library.)
+ *   Same layer, x_dev, M, y_dev, stream and results as mpq_linear.  The
+ *   scratch is one static device array of MPQ_NOALLOC_SCRATCH_BYTES
+ *   (6 MiB) inside the library, held by every GPU that loads the library
+ *   until the process exits; no cudaMalloc/cudaFree or other allocating
+ *   call is made.  Sizes whose workspace (mpq_linear_workspace_size) would
+ *   exceed it return MPQ_ERR_WORKSPACE.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls share the one array, which keeps the last call's contents
+ *   (the parts that must start at zero are cleared by each call): calls
+ *   that overlap on the GPU -- on different streams, or from different
+ *   threads -- race and give wrong results.  Serialize them.
+ *   Device-side errors go to the array's error word, which mpq_check cannot
+ *   see; host-side errors are returned as for mpq_linear. */
+#define MPQ_NOALLOC_SCRATCH_BYTES (6u << 20)
+mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t M,
+                              float* y_dev, void* stream);
+
 /* Synchronizes `stream` and returns the device error word stored in `ws` by
  * the last mpq_pack / mpq_linear on that workspace (MPQ_OK if none). */
 mpq_status mpq_check(const void* ws, void* stream);
