@@ -314,9 +314,9 @@ def run_gpu(args):
     from block_wise_mixed_b200 import synth
 
     peaks, peak_src = load_peaks()
-    layer = synth.config_layer(HEADLINE_CFG, 0)
-    M = 1
     if args.quick:
+        layer = synth.config_layer(args.cfg, args.proj)
+        M = args.M
         # the timed loop only (for profiler captures of the same command)
         r = time_layer(mpq, layer, M, args.steps, args.warmup, world, device, soak_s=0.0,
                        quick=True)
@@ -327,6 +327,8 @@ def run_gpu(args):
             import torch.distributed as dist
             dist.destroy_process_group()
         return
+    layer = synth.config_layer(HEADLINE_CFG, 0)
+    M = 1
     sampler = ClockSampler(local)
     r = time_layer(mpq, layer, M, args.steps, args.warmup, world, device, sampler=sampler)
 
@@ -362,12 +364,115 @@ def run_gpu(args):
         res["cpu_baseline"] = oracle_baseline(layer, xb, min_seconds=args.cpu_seconds)
     if args.extra and rank == 0:
         res["extra"] = run_extra(mpq, args, device, peaks)
+        res["extra"]["tensor_core_llama3_8b_layer"] = run_tensor_core(mpq, args, device, peaks)
+        res["extra"]["pack_llama3_8b_layer"] = run_pack(mpq, device, peaks)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+def time_prefill(mpq, L, M, steps, device):
+    """Tensor-core path: kernel time (events around the main kernel) and the
+    whole mpq_linear step for one layer at M tokens."""
+    import torch
+    from block_wise_mixed_b200 import synth
+    W = torch.from_numpy(L.W.view(np.int16)).to(device)
+    P = mpq.pack(W, L.bits, L.row_perm, L.col_perm)
+    del W
+    lay = P.layout
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    per_rep = lay.codes_bytes + 4 * lay.n_sz
+    R = int(max(2, min(64, np.ceil(4 * l2 / max(per_rep, 1)))))
+    reps = build_replicas(mpq, P, R)
+    x = torch.from_numpy(synth.make_x(synth.seed_of(98, 0), M, L.K).view(np.int16)).to(device)
+    y = torch.empty((M, L.N), dtype=torch.float32, device=device)
+    ws = torch.empty(mpq.linear_workspace_size(P, M), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for i in range(3):
+        mpq.linear(reps[i % R], x, y, ws)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream); b.record(stream)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s_ in range(steps):
+        mpq.linear_timed(reps[s_ % R], x, y, ws, evs[s_][0], evs[s_][1])
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    k_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    step_ms = e0.elapsed_time(e1) / steps
+    f0 = float((L.bits == 0).mean())
+    flops = 2.0 * M * L.N * L.K * (1.0 - f0)
+    del reps
+    torch.cuda.empty_cache()
+    return dict(name=L.name, N=L.N, K=L.K, M=M, f0=f0, kernel_us=k_ms * 1e3, step_us=step_ms * 1e3,
+                flops=flops, dense_flops=2.0 * M * L.N * L.K)
+
+
+def time_pack(mpq, L, device, reps=3):
+    """mpq_pack of one layer: GPU time with events (host planning excluded
+    from the events but included in the wall time)."""
+    import torch
+    W = torch.from_numpy(L.W.view(np.int16)).to(device)
+    mpq.pack(W, L.bits, L.row_perm, L.col_perm)      # warm-up
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    ts, walls = [], []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        a.record(stream)
+        P = mpq.pack(W, L.bits, L.row_perm, L.col_perm, check=False)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        walls.append(time.perf_counter() - t0)
+        ts.append(a.elapsed_time(b))
+    lay = P.layout
+    nbytes = 2 * L.N * L.K + lay.codes_bytes + 4 * lay.n_sz
+    return dict(name=L.name, gpu_us=float(np.median(ts)) * 1e3, wall_ms=float(np.median(walls)) * 1e3,
+                bytes=nbytes)
+
+
+def run_tensor_core(mpq, args, device, peaks, which=None):
+    """Llama-3-8B layer at M = 512 and 2048 on the tensor-core path."""
+    from block_wise_mixed_b200 import synth
+    projs = range(7) if which is None else which
+    out = {}
+    for M in (512, 2048):
+        tot_flops = tot_us = 0.0
+        per = {}
+        for proj in projs:
+            L = synth.config_layer(5, proj)
+            r = time_prefill(mpq, L, M, 10, device)
+            tot_flops += r["flops"]
+            tot_us += r["kernel_us"]
+            per[L.name] = {"kernel_us": round(r["kernel_us"], 1), "step_us": round(r["step_us"], 1),
+                           "TFLOPs": round(r["flops"] / (r["kernel_us"] * 1e-6) / 1e12, 1)}
+        tf = tot_flops / (tot_us * 1e-6) / 1e12
+        out["M%d" % M] = {"layer_kernel_us": round(tot_us, 1), "TFLOPs": round(tf, 1),
+                          "frac_burst": round(tf / peaks["bf16_tflops"], 4),
+                          "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                          "projections": per}
+    return out
+
+
+def run_pack(mpq, device, peaks):
+    from block_wise_mixed_b200 import synth
+    tot_us = tot_bytes = 0.0
+    per = {}
+    for proj in range(7):
+        L = synth.config_layer(5, proj)
+        r = time_pack(mpq, L, device)
+        tot_us += r["gpu_us"]
+        tot_bytes += r["bytes"]
+        per[L.name] = {"gpu_us": round(r["gpu_us"], 1), "wall_ms": round(r["wall_ms"], 2)}
+    gbs = tot_bytes / (tot_us * 1e-6) / 1e9
+    return {"layer_gpu_us": round(tot_us, 1), "GBps": round(gbs, 1),
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "projections": per}
 
 
 def run_extra(mpq, args, device, peaks):
@@ -440,6 +545,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",
                     help="timed loop only, no soak/e2e/CPU baseline (for ncu)")
+    ap.add_argument("--cfg", type=int, default=HEADLINE_CFG, help="workload for --quick")
+    ap.add_argument("--proj", type=int, default=0, help="projection for --quick")
+    ap.add_argument("--M", type=int, default=1, help="tokens for --quick")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -1,0 +1,411 @@
+// k_prefill.cuh -- tensor-core (tcgen05 / TMEM) mixed-precision GEMM for
+// larger token counts.
+//
+// D[i][m] = sum_k w_hat'[i][k] * x'[m][k] for a tile of 128 weight rows
+// (two 64-row block rows) and 128 tokens; y[m][row_perm[i]] = D * tok_scale[m].
+// The blocks' dequantization is the RTN of the ScaleBITS summary ("Approach",
+// "Key results"); TileQuant's abstract describes the same split -- compact
+// per-tile buffers expanded next to the 16-bit tensor-core computation.
+//
+// Roles (10 warps):
+//   warp 0     producer: 1-D bulk copies of the two blocks' payloads and
+//              scales/zeros per 128-wide k block into a ring, and the x' tile
+//              (TMA tensor copy, 128B swizzle) into the operand stage.
+//   warp 1     allocates TMEM and issues tcgen05.mma (one elected thread).
+//   warps 2-9  dequantize: each thread expands half of one weight row's
+//              128 codes into fp16 w_hat = (q - z) * s, written straight
+//              into the K-major 128B-swizzled shared-memory A operand; after
+//              the last k block they read the fp32 accumulator out of TMEM
+//              and write y.
+// A k block whose two blocks are both 0-bit is skipped by every role (no
+// bytes, no MMA); a 0-bit block next to a non-zero one contributes zero rows.
+// The operands are fp16 (A = dequantized weights, B = x' scaled per token by a
+// power of two); accumulation is fp32 in TMEM.
+//
+// The x' layout (written by k_xprep, XP_PREFILL) permutes each 128-column
+// group so that MMA k = 2*(4i+j)+h holds column 8i+j+4h: the extraction emits
+// the pair (8i+j, 8i+j+4) in one register, so a group of 8 codes becomes one
+// 16-byte chunk of A.
+//
+// All waits are bounded (MPQ_ERR_TIMEOUT); the kernel then winds down.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "k_decode.cuh"   // code extraction helpers (ext1/2/4/8, *_hi)
+
+namespace mpq {
+
+constexpr int PF_WARPS = 10;
+constexpr int PF_THREADS = PF_WARPS * 32;
+constexpr int PF_DQ_WARPS = 8;
+constexpr int PF_BM = 128;       // weight rows per tile (2 block rows)
+constexpr int PF_BN = 128;       // tokens per tile
+constexpr int PF_AB_STAGES = 2;
+constexpr int PF_C_STAGES = 3;
+constexpr int PF_A_BYTES = PF_BM * 256;           // 128 rows x 128 fp16
+constexpr int PF_B_BYTES = PF_BN * 256;           // 128 tokens x 128 fp16
+constexpr int PF_C_BYTES = 2 * 8192 + 4 * 128;    // two payloads + 2 x (scales, zeros)
+constexpr uint32_t PF_TMEM_COLS = 128;
+
+struct PrefillSmem {
+    uint8_t a[PF_AB_STAGES][PF_A_BYTES];   // 1024-aligned (offset 0)
+    uint8_t b[PF_AB_STAGES][PF_B_BYTES];
+    uint8_t c[PF_C_STAGES][PF_C_BYTES];
+    uint64_t full_ab[PF_AB_STAGES];
+    uint64_t empty_ab[PF_AB_STAGES];
+    uint64_t full_c[PF_C_STAGES];
+    uint64_t empty_c[PF_C_STAGES];
+    uint64_t d_full;
+    uint32_t tmem_base;
+    volatile int abort_flag;
+    // per tile: code_off, sz_off, bits of the two block rows, KB entries each
+};
+
+struct PrefillParams {
+    const uint8_t* codes;
+    const mpq_block* table;
+    const uint16_t* scales;
+    const uint16_t* zeros;
+    const int32_t* row_perm;
+    const float* tok_scale;   // [M]
+    float* y;                 // [M][N]
+    uint32_t* err;
+    int N, K, NB, KB, M;
+    int tiles_n;              // ceil(NB / 2)
+};
+
+__device__ __forceinline__ uint64_t umma_smem_desc_sw128(uint32_t saddr) {
+    // K-major, 128-byte swizzle: 8-row groups 1024 B apart (SBO), LBO unused
+    // (1), descriptor version 1, layout type 2 = SWIZZLE_128B.
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// kind::f16 instruction descriptor: D = F32, A = B = F16, both K-major.
+__device__ __forceinline__ constexpr uint32_t umma_idesc_f16(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's TMEM lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Offset of the 16-byte chunk holding K elements 8*kc..8*kc+7 of row r in a
+// 128-row x 128-K tile stored K-major with 128B swizzle (two 64-K halves).
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int kc) {
+    return (uint32_t)((kc >> 3) * (PF_BM * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                      (((kc & 7) ^ (r & 7)) << 4));
+}
+
+// Dequantizes groups [g0, g0+8) (8 codes each) of row rr of one block of
+// width B into the A tile row r: w_hat = (q - z) * s in fp16.
+template <int B>
+__device__ __forceinline__ void dequant_row_half(const uint8_t* payload, const __half* scz, int rr,
+                                                 int g0, uint8_t* a_tile, int r) {
+    constexpr int P0 = (B == 3) ? 2 : (B == 5 || B == 6) ? 4 : B;
+    constexpr int P1 = (B == 3 || B == 5) ? 1 : (B == 6) ? 2 : 0;
+    const __half sh = scz[rr];
+    const uint32_t z2 = __byte_perm((uint32_t)__half_as_ushort(scz[64 + rr]), 0u, 0x1010);
+    const __half2 s2 = __half2half2(sh);
+    uint32_t k[4];
+    zero_consts<P0>(z2, k);
+    // this half-row's bytes of each piece: groups g0..g0+7 = codes 8*g0 .. 8*g0+63
+    const uint8_t* lo = payload + rr * 16 * P0 + (g0 * 8 * P0) / 8;
+    uint32_t d[2 * P0];   // 64 codes of P0 bits = 8*P0 bytes = 2*P0 words
+#pragma unroll
+    for (int q = 0; q < 2 * P0; q += (P0 >= 2 ? 2 : 1)) {
+        if (P0 >= 2) {
+            uint2 v = *reinterpret_cast<const uint2*>(lo + 4 * q);
+            d[q] = v.x; d[q + 1] = v.y;
+        } else {
+            d[q] = *reinterpret_cast<const uint32_t*>(lo + 4 * q);
+        }
+    }
+    uint32_t e[P1 > 0 ? 2 * P1 : 1];
+    if (P1 > 0) {
+        const uint8_t* hi = payload + 64 * 16 * P0 + rr * 16 * P1 + (g0 * 8 * P1) / 8;
+#pragma unroll
+        for (int q = 0; q < 2 * P1; ++q) e[q] = *reinterpret_cast<const uint32_t*>(hi + 4 * q);
+    }
+#pragma unroll
+    for (int gi = 0; gi < 8; ++gi) {
+        uint32_t o[4];
+        if (P0 == 4) {
+            ext4(d[gi], k[0], k[1], o);
+        } else if (P0 == 8) {
+            ext8(d[2 * gi], d[2 * gi + 1], k[0], o);
+        } else if (P0 == 2) {
+            ext2(d[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, k, o);
+        } else {
+            const int bi = gi & 3;
+            ext1(d[gi >> 2], bi | (4 << 4) | (bi << 8) | (4 << 12), k, o);
+        }
+        if (P1 > 0) {
+            uint32_t h[4];
+            if (P1 == 1) {
+                const int bi = gi & 3;
+                ext1_hi<P0>(e[gi >> 2], bi | (4 << 4) | (bi << 8) | (4 << 12), h);
+            } else {
+                ext2_hi(e[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, h);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = h2_bits(__hadd2(bits_h2(o[j]), bits_h2(h[j])));
+        }
+        uint4 w;
+        w.x = h2_bits(__hmul2(bits_h2(o[0]), s2));
+        w.y = h2_bits(__hmul2(bits_h2(o[1]), s2));
+        w.z = h2_bits(__hmul2(bits_h2(o[2]), s2));
+        w.w = h2_bits(__hmul2(bits_h2(o[3]), s2));
+        *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + gi)) = w;
+    }
+}
+
+__global__ void __launch_bounds__(PF_THREADS, 1)
+k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // the operand tiles need 1024-byte alignment (128B swizzle atoms)
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(base);
+    uint32_t* tab = reinterpret_cast<uint32_t*>(base + sizeof(PrefillSmem));  // [2][KB][3]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int KB = p.KB;
+    const int tile_n = blockIdx.x % p.tiles_n;
+    const int tile_m = blockIdx.x / p.tiles_n;
+    const int nb0 = 2 * tile_n;
+    const int m0 = tile_m * PF_BN;
+
+    // stage this tile's table entries: tab[(h*KB + kb)*3 + {0,1,2}]
+    for (int i = tid; i < 2 * KB; i += PF_THREADS) {
+        const int h = i / KB, kb = i % KB;
+        const int nb = nb0 + h;
+        uint32_t co = 0, so = 0, bits = 0;
+        if (nb < p.NB) {
+            const mpq_block e = p.table[(size_t)nb * KB + kb];
+            co = e.code_off; so = e.sz_off; bits = e.bits;
+        }
+        tab[3 * i] = co; tab[3 * i + 1] = so; tab[3 * i + 2] = bits;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < PF_AB_STAGES; ++s) {
+            mbar_init(&S.full_ab[s], 1 + PF_DQ_WARPS);
+            mbar_init(&S.empty_ab[s], 1);
+        }
+        for (int s = 0; s < PF_C_STAGES; ++s) {
+            mbar_init(&S.full_c[s], 1);
+            mbar_init(&S.empty_c[s], PF_DQ_WARPS);
+        }
+        mbar_init(&S.d_full, 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&S.tmem_base)),
+                     "r"(PF_TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = S.tmem_base;
+
+    auto timed_out = [&]() {
+        set_error(p.err, MPQ_ERR_TIMEOUT);
+        S.abort_flag = 1;
+    };
+    auto bits_of = [&](int h, int kb) -> uint32_t { return tab[3 * (h * KB + kb) + 2]; };
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        pdl_wait();   // x' and tok_scale come from the prologue kernel
+        if (lane == 0) {
+            int a = 0;
+            for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
+                const uint32_t b0 = bits_of(0, kb), b1 = bits_of(1, kb);
+                if ((b0 | b1) == 0) continue;
+                const int sc = a % PF_C_STAGES;
+                const uint32_t pc = (uint32_t)(a / PF_C_STAGES) & 1u;
+                if (!mbar_wait_bounded(&S.empty_c[sc], pc ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
+                uint32_t bytes = (b0 ? 1024u * b0 + 256u : 0u) + (b1 ? 1024u * b1 + 256u : 0u);
+                mbar_arrive_expect_tx(&S.full_c[sc], bytes);
+                uint8_t* cst = S.c[sc];
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t b = h ? b1 : b0;
+                    if (!b) continue;
+                    const uint32_t co = tab[3 * (h * KB + kb)], so = tab[3 * (h * KB + kb) + 1];
+                    bulk_g2s(cst + h * 8192, p.codes + co, 1024u * b, &S.full_c[sc]);
+                    bulk_g2s(cst + 16384 + h * 256, p.scales + so, 128u, &S.full_c[sc]);
+                    bulk_g2s(cst + 16384 + h * 256 + 128, p.zeros + so, 128u, &S.full_c[sc]);
+                }
+                const int s = a % PF_AB_STAGES;
+                const uint32_t ps = (uint32_t)(a / PF_AB_STAGES) & 1u;
+                if (!mbar_wait_bounded(&S.empty_ab[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
+                mbar_arrive_expect_tx(&S.full_ab[s], (uint32_t)PF_B_BYTES);
+                tma_load_2d(S.b[s], &tmap_x, kb * 128, m0, &S.full_ab[s]);
+                tma_load_2d(S.b[s] + PF_BN * 128, &tmap_x, kb * 128 + 64, m0, &S.full_ab[s]);
+                ++a;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ----------------------------
+        const uint32_t idesc = umma_idesc_f16(PF_BM, PF_BN);
+        int a = 0;
+        if (lane == 0) {
+            for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
+                if ((bits_of(0, kb) | bits_of(1, kb)) == 0) continue;
+                const int s = a % PF_AB_STAGES;
+                const uint32_t ps = (uint32_t)(a / PF_AB_STAGES) & 1u;
+                if (!mbar_wait_bounded(&S.full_ab[s], ps, DEC_WAIT_NS)) { timed_out(); break; }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(S.a[s]), b_base = smem_u32(S.b[s]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (uint32_t)((kk >> 2) * (PF_BM * 128) + (kk & 3) * 32);
+                    const uint32_t offb = (uint32_t)((kk >> 2) * (PF_BN * 128) + (kk & 3) * 32);
+                    umma_f16_ss(tmem_d, umma_smem_desc_sw128(a_base + off),
+                                umma_smem_desc_sw128(b_base + offb), idesc,
+                                (a > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&S.empty_ab[s]);
+                ++a;
+            }
+            if (a > 0) umma_commit(&S.d_full);
+            else mbar_arrive(&S.d_full);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------- dequantize, then epilogue ----------------------
+        const int dw = warp - 2;                 // 0..7
+        const int quad = warp & 3;               // TMEM lane quadrant of this warp
+        const int half = dw >> 2;                // which 64 K / 64 tokens this warp takes
+        const int r = quad * 32 + lane;          // weight row in the tile (= TMEM lane)
+        const int h = r >> 6, rr = r & 63;
+        int a = 0;
+        bool any = false;
+        for (int kb = 0; kb < KB; ++kb) {
+            const uint32_t b0 = bits_of(0, kb), b1 = bits_of(1, kb);
+            if ((b0 | b1) == 0) continue;
+            any = true;
+            if (S.abort_flag) break;
+            const int sc = a % PF_C_STAGES;
+            const uint32_t pc = (uint32_t)(a / PF_C_STAGES) & 1u;
+            const int s = a % PF_AB_STAGES;
+            const uint32_t ps = (uint32_t)(a / PF_AB_STAGES) & 1u;
+            bool ok = mbar_wait_bounded(&S.full_c[sc], pc, DEC_WAIT_NS);
+            ok = ok && mbar_wait_bounded(&S.empty_ab[s], ps ^ 1u, DEC_WAIT_NS);
+            if (!__all_sync(0xffffffffu, ok)) { if (lane == 0) timed_out(); break; }
+            const uint32_t b = h ? b1 : b0;
+            uint8_t* a_tile = S.a[s];
+            const uint8_t* cst = S.c[sc];
+            const __half* scz = reinterpret_cast<const __half*>(cst + 16384 + h * 256);
+            const int g0 = half * 8;
+            switch (b) {
+                case 0: {
+                    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int gi = 0; gi < 8; ++gi)
+                        *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + gi)) = zero;
+                    break;
+                }
+                case 1: dequant_row_half<1>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 2: dequant_row_half<2>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 3: dequant_row_half<3>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 4: dequant_row_half<4>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 5: dequant_row_half<5>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 6: dequant_row_half<6>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                default: dequant_row_half<8>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+            }
+            fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&S.full_ab[s]);
+                mbar_arrive(&S.empty_c[sc]);
+            }
+            ++a;
+        }
+        // epilogue: this warp's 32 rows x its 64 tokens
+        pdl_wait();   // tok_scale comes from the prologue kernel
+        bool ok = S.abort_flag ? false : mbar_wait_bounded(&S.d_full, 0u, DEC_WAIT_NS);
+        if (!__all_sync(0xffffffffu, ok) && !S.abort_flag && lane == 0) timed_out();
+        tc_fence_after();
+        const int i = nb0 * 64 + r;
+        const bool row_ok = i < p.N;
+        const int n = row_ok ? (p.row_perm ? p.row_perm[i] : i) : 0;
+        for (int cc = 0; cc < 2; ++cc) {
+            const int col0 = half * 64 + cc * 32;
+            float v[32];
+            if (any && ok) {
+                tmem_ld32(tmem_d + ((uint32_t)(quad * 32) << 16) + (uint32_t)col0, v);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            }
+            if (row_ok) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int m = m0 + col0 + j;
+                    if (m < p.M) p.y[(size_t)m * p.N + n] = v[j] * p.tok_scale[m];
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d),
+                     "r"(PF_TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace mpq

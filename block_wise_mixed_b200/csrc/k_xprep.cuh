@@ -14,16 +14,24 @@
 //               32t+8i+j+4) of that block column: exactly the B fragment of
 //               mma.m16n8k16 that the decode kernel pairs with its code
 //               extraction order.
-//   XP_ROWMAJOR: [M][K] half, K contiguous (the tensor-core kernel's A/B tile
-//               source).
-// Block 0 also clears the workspace error word and the per-block-row
-// counters of the decode kernel's fix-up.
+//   XP_PREFILL: [M][K] half, K contiguous, each 128-column group permuted so
+//               that position 2*(4i+j)+h holds column 8i+j+4h -- the order in
+//               which the tensor-core kernel's dequantization emits weights.
+// Block 0 also clears the workspace error word.
+//
+// k_xprep_decode (below) is the small-batch variant: one warp per (block
+// column kb, token m) and no row-wide reduction.  Each 128-column slice gets
+// its own power of two 2^e (from the slice's largest magnitude), stored with
+// the slice; the decode kernel folds 2^-e into its per-group fp32 scale.
+// Layout [KB][M][272 bytes]: 4 quad lanes x 16 half2 in the mma B-fragment
+// order of XP_DECODE, then the fp32 factor 2^-e and 12 bytes of padding.
+// It also clears the decode kernel's per-block-row counters.
 #pragma once
 #include "common.cuh"
 
 namespace mpq {
 
-enum XprepLayout { XP_DECODE = 0, XP_ROWMAJOR = 1 };
+enum XprepLayout { XP_DECODE = 0, XP_PREFILL = 1 };
 
 struct XprepParams {
     const uint16_t* x;         // bf16 bits, M x K
@@ -46,7 +54,8 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
     const int m = blockIdx.x, tid = threadIdx.x, K = p.K;
     if (m == 0) {
         if (tid == 0 && p.err) *p.err = 0u;
-        for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
+        if (p.counters)
+            for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
     }
     const uint16_t* xr = p.x + (size_t)m * K;
     // 1. amax over the row (order-free, so read it unpermuted, 8 values per load)
@@ -99,8 +108,75 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
         (void)KB;
     } else {
         __half2* out = reinterpret_cast<__half2*>(p.xq + (size_t)m * K);
-        for (int c2 = tid; c2 < K / 2; c2 += XPREP_THREADS)
-            out[c2] = __halves2half2(__float2half_rn(load(2 * c2)), __float2half_rn(load(2 * c2 + 1)));
+        for (int c2 = tid; c2 < K / 2; c2 += XPREP_THREADS) {
+            const int kb = c2 >> 6, r = c2 & 63, i = r >> 2, j = r & 3;
+            const int col = kb * 128 + 8 * i + j;
+            out[c2] = __halves2half2(__float2half_rn(load(col)), __float2half_rn(load(col + 4)));
+        }
+    }
+}
+
+constexpr int XQD_SLICE = 272;   // bytes per (kb, token) slice
+
+__global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int KB = p.K / 128;
+    if (blockIdx.x == 0) {
+        if (tid == 0 && p.err) *p.err = 0u;
+        if (p.counters)
+            for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
+    }
+    const int item = blockIdx.x * (XPREP_THREADS / 32) + (tid >> 5);   // = kb * M + m
+    if (item >= KB * p.M) return;
+    const int kb = item / p.M, m = item % p.M;
+    const uint16_t* xr = p.x + (size_t)m * p.K;
+    // lane holds columns 4*lane .. 4*lane+3 of the slice
+    float v[4];
+    const int c0 = kb * 128 + 4 * lane;
+    if (p.col_perm) {
+        const int4 cp = *reinterpret_cast<const int4*>(p.col_perm + c0);
+        v[0] = __uint_as_float((uint32_t)xr[cp.x] << 16);
+        v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
+        v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
+        v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
+    } else {
+        const uint2 raw = *reinterpret_cast<const uint2*>(xr + c0);
+        v[0] = __uint_as_float(raw.x << 16);
+        v[1] = __uint_as_float(raw.x & 0xffff0000u);
+        v[2] = __uint_as_float(raw.y << 16);
+        v[3] = __uint_as_float(raw.y & 0xffff0000u);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+        const float a = fabsf(v[e4]);
+        amax = (a > amax || a != a) ? a : amax;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, amax, off);
+        amax = (o > amax || o != o) ? o : amax;
+    }
+    int e = 0;
+    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -126), 126);
+    // pair (8i+j, 8i+j+4): columns 8i..8i+3 sit in lane 2i', 8i+4..8i+7 in lane 2i'+1
+    float w[4];
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) w[e4] = __shfl_down_sync(0xffffffffu, v[e4], 1);
+    uint8_t* slice = reinterpret_cast<uint8_t*>(p.xq) + (size_t)item * XQD_SLICE;
+    if ((lane & 1) == 0) {
+        // this lane's 8 columns are 8*(lane/2) .. +7 of the slice: quad lane
+        // t = lane/8, group i = (lane/2) % 4, registers 4i .. 4i+3
+        uint4 out;
+        uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = h2_bits(__halves2half2(__float2half_rn(ldexpf(v[j], e)), __float2half_rn(ldexpf(w[j], e))));
+        *reinterpret_cast<uint4*>(slice + (lane >> 1) * 16) = out;
+    }
+    if (lane == 0) {
+        *reinterpret_cast<float4*>(slice + 256) = make_float4(ldexpf(1.f, -e), 0.f, 0.f, 0.f);
     }
 }
 

@@ -1,6 +1,8 @@
 // mpq_api.cu -- the C ABI of libmpq (declared in include/mpq.h): host-side
 // validation, the plan (segment offsets, block table, decode schedule) and
 // the kernel launches.  The library allocates no device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -13,15 +15,17 @@
 #include "common.cuh"
 #include "k_decode.cuh"
 #include "k_pack.cuh"
+#include "k_prefill.cuh"
 #include "k_xprep.cuh"
 
 using namespace mpq;
 
 namespace {
 
-constexpr int kMaxUnits = 444;          // 3 decode CTAs on each of 148 SMs
+constexpr int kMaxUnits = 592;          // 4 decode CTAs on each of 148 SMs
 constexpr uint64_t kMinUnitBits = 8;    // >= 8 KiB of codes per decode unit
 constexpr int kMaxDecodeTokens = 8;     // tokens per decode launch
+constexpr int kDecodeMaxM = 16;         // larger batches take the tensor-core kernel
 constexpr int kPackRowsPerCta = 16;
 
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -121,7 +125,8 @@ LinearWs carve_linear(void* ws, const mpq_layer* layer, int32_t M) {
     w.tok_scale = reinterpret_cast<float*>(base + off);
     off += round256((size_t)M * 4);
     w.xq = reinterpret_cast<__half*>(base + off);
-    off += round256((size_t)M * layer->K * 2);
+    // decode: [KB][M][XQD_SLICE]; tensor-core path: [M][K] fp16 (smaller)
+    off += round256((size_t)(layer->K / 128) * M * XQD_SLICE);
     w.partial = reinterpret_cast<float*>(base + off);
     off += round256((size_t)2 * layer->n_units * 64 * 8 * 4);
     w.bytes = off;
@@ -148,6 +153,38 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
     return e;
 }
 std::atomic<uint64_t> g_decode_attr{0};
+std::atomic<uint64_t> g_prefill_attr{0};
+
+// cuTensorMapEncodeTiled from the driver, looked up through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// 2-D fp16 [rows][K] tensor, 64 x box_rows boxes, 128-byte swizzle.
+bool make_tmap_fp16(CUtensorMap* map, const void* ptr, int K, int rows, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+size_t prefill_smem_bytes(int KB) {
+    return sizeof(PrefillSmem) + 1024 + (size_t)2 * KB * 12;
+}
 
 }  // namespace
 
@@ -246,6 +283,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int NB = layer->N / 64, KB = layer->K / 128;
 
+    const bool use_tc = M > kDecodeMaxM;
     XprepParams xp{};
     xp.x = static_cast<const uint16_t*>(x_dev);
     xp.col_perm = layer->col_perm;
@@ -256,9 +294,57 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     xp.err = w.err;
     xp.M = M;
     xp.K = layer->K;
-    k_xprep<XP_DECODE><<<M, XPREP_THREADS, 0, s>>>(xp);
+    if (use_tc) {
+        xp.counters = nullptr;
+        k_xprep<XP_PREFILL><<<M, XPREP_THREADS, 0, s>>>(xp);
+    } else {
+        const int items = KB * M, per = XPREP_THREADS / 32;
+        k_xprep_decode<<<(items + per - 1) / per, XPREP_THREADS, 0, s>>>(xp);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
+
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    if (use_tc) {
+        const size_t smem = prefill_smem_bytes(KB);
+        if (smem > 227 * 1024) return MPQ_ERR_SHAPE;
+        e = ensure_smem_attr(k_prefill, 227 * 1024, g_prefill_attr);   // the sm_100 maximum
+        if (e != cudaSuccess) return MPQ_ERR_CUDA;
+        CUtensorMap tmap;
+        if (!make_tmap_fp16(&tmap, w.xq, layer->K, M, PF_BN)) return MPQ_ERR_CUDA;
+        PrefillParams pp{};
+        pp.codes = static_cast<const uint8_t*>(layer->codes);
+        pp.table = layer->table;
+        pp.scales = layer->scales;
+        pp.zeros = layer->zeros;
+        pp.row_perm = layer->row_perm;
+        pp.tok_scale = w.tok_scale;
+        pp.y = y_dev;
+        pp.err = w.err;
+        pp.N = layer->N;
+        pp.K = layer->K;
+        pp.NB = NB;
+        pp.KB = KB;
+        pp.M = M;
+        pp.tiles_n = (NB + 1) / 2;
+        const int tiles_m = (M + PF_BN - 1) / PF_BN;
+        cudaLaunchConfig_t pc{};
+        pc.gridDim = dim3((unsigned)(pp.tiles_n * tiles_m));
+        pc.blockDim = dim3(PF_THREADS);
+        pc.dynamicSmemBytes = smem;
+        pc.stream = s;
+        pc.attrs = pdl;
+        pc.numAttrs = 1;
+        if (ev_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s) != cudaSuccess)
+            return MPQ_ERR_CUDA;
+        e = cudaLaunchKernelEx(&pc, k_prefill, pp, tmap);
+        if (e != cudaSuccess) return MPQ_ERR_CUDA;
+        if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
+            return MPQ_ERR_CUDA;
+        return MPQ_OK;
+    }
 
     e = ensure_smem_attr(k_decode, (int)sizeof(DecSmem), g_decode_attr);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
@@ -270,7 +356,6 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     dp.zeros = layer->zeros;
     dp.row_perm = layer->row_perm;
     dp.xq = reinterpret_cast<const uint8_t*>(w.xq);
-    dp.tok_scale = w.tok_scale;
     dp.y = y_dev;
     dp.partial = w.partial;
     dp.counters = w.counters;
