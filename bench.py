@@ -233,6 +233,14 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
             mpq.linear(reps[i % R], x, y, ws)
             i += 1
         torch.cuda.synchronize(device)
+    # the timed steps run as one CUDA graph (launch overhead of the host
+    # binding is not part of the device time, as in graph-launched decoding)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for s_ in range(steps):
+            mpq.linear(reps[s_ % R], x, y, ws)
+    graph.replay()
+    torch.cuda.synchronize(device)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -240,8 +248,7 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for s in range(steps):
-        mpq.linear(reps[s % R], x, y, ws)
+    graph.replay()
     e1.record(stream)
     torch.cuda.synchronize(device)
     clocks = sampler.stop() if sampler else None
@@ -249,18 +256,22 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     ms_step = reduce_max_over_ranks(ms_total, world, device) / steps
     nbytes = algorithmic_bytes(L.N, L.K, M, lay.codes_bytes, lay.n_sz, T,
                                L.row_perm is not None, L.col_perm is not None)
+    del graph
     if quick:
         return dict(N=L.N, K=L.K, M=M, bytes=nbytes, ms_step=ms_step, replicas=R)
 
-    # main-kernel time alone, events recorded by the library around it
+    # main-kernel time alone: events recorded by the library around it.  A
+    # spin kernel first holds the GPU while the host enqueues every call, so
+    # the calls run back to back and the events see device time only.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
     for a, b in evs:        # torch creates the CUDA events on first record
         a.record(stream)
         b.record(stream)
     torch.cuda.synchronize(device)
-    for s in range(steps):
-        mpq.linear_timed(reps[s % R], x, y, ws, evs[s][0], evs[s][1])
+    torch.cuda._sleep(int(2e6 + 4e4 * steps))   # ~1 ms + 20 us per enqueued call
+    for s_ in range(steps):
+        mpq.linear_timed(reps[s_ % R], x, y, ws, evs[s_][0], evs[s_][1])
     torch.cuda.synchronize(device)
     k_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
@@ -398,6 +409,7 @@ def time_prefill(mpq, L, M, steps, device):
         a.record(stream); b.record(stream)
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(2e6 + 4e4 * steps))   # the host enqueues ahead of the GPU
     e0.record(stream)
     for s_ in range(steps):
         mpq.linear_timed(reps[s_ % R], x, y, ws, evs[s_][0], evs[s_][1])
