@@ -332,7 +332,8 @@ def run_gpu(args):
         r = time_layer(mpq, layer, M, args.steps, args.warmup, world, device, soak_s=0.0,
                        quick=True)
         if rank == 0:
-            print(json.dumps({"quick": True, "ms_per_step": r["ms_step"],
+            print(json.dumps({"quick": True, "cfg": args.cfg, "proj": args.proj, "M": M,
+                              "N": layer.N, "K": layer.K, "us_per_step": r["ms_step"] * 1e3,
                               "GBps": r["bytes"] / (r["ms_step"] * 1e-3) / 1e9}), flush=True)
         if world > 1:
             import torch.distributed as dist

@@ -37,7 +37,7 @@ class Block(ctypes.Structure):
 class Layout(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("NB", ctypes.c_int32),
                 ("KB", ctypes.c_int32), ("n_units", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("codes_bytes", ctypes.c_uint64),
+                ("sched_words", ctypes.c_int32), ("codes_bytes", ctypes.c_uint64),
                 ("n_sz", ctypes.c_uint64), ("bit_total", ctypes.c_uint64),
                 ("seg_off", ctypes.c_uint64 * 9), ("seg_bytes", ctypes.c_uint64 * 9)]
 
@@ -70,6 +70,7 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
         L.mpq_plan.argtypes = [i32, i32, P, ctypes.POINTER(Layout)]
+        L.mpq_plan_schedule.argtypes = [ctypes.POINTER(Layout), P, P]
         L.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
         L.mpq_pack_workspace_size.restype = sz
         L.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
@@ -119,6 +120,14 @@ def plan(N: int, K: int, bits: np.ndarray) -> Layout:
     return L
 
 
+def plan_schedule(L: Layout, bits: np.ndarray) -> np.ndarray:
+    """mpq_plan_schedule: the decode schedule mpq_pack stores (host only)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint8).reshape(-1)
+    out = np.zeros(L.sched_words, np.uint32)
+    _raise(lib().mpq_plan_schedule(ctypes.byref(L), _np_ptr(bits), _np_ptr(out)), "mpq_plan_schedule")
+    return out
+
+
 @dataclass
 class PackedLayer:
     """A packed layer in device memory (torch tensors) plus its C view."""
@@ -151,7 +160,7 @@ def alloc_layer(L: Layout, device, has_row_perm: bool, has_col_perm: bool) -> Pa
     T = L.NB * L.KB
     codes = buf(L.codes_bytes)
     table = buf(T * 16)
-    sched = buf((L.n_units + 1) * 4)
+    sched = buf(L.sched_words * 4)
     scales = buf(2 * L.n_sz)
     zeros = buf(2 * L.n_sz)
     rp = torch.empty(L.N, dtype=torch.int32, device=device) if has_row_perm else None

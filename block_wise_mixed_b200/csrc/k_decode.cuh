@@ -3,42 +3,70 @@
 // y'[m][i] = sum_kb s[i,kb] * sum_{j in kb} x'[m][j] * (q[i][j] - z[i,kb])
 // (the blocks' RTN dequantization, ScaleBITS summary "Approach" / "Key
 // results"; 0-bit blocks are skipped -- they hold no bytes), then
-// y[m][row_perm[i]] = y'[m][i] * tok_scale[m].
+// y[m][row_perm[i]] = y'[m][i].
 //
-// Work split.  The table's blocks are cut, at pack time, into `n_units`
-// row-major runs of about equal code bytes (sched); one CTA per run.  A CTA
-// is 4 warps; the non-zero blocks of its run are dealt round-robin to the
-// warps, and each warp streams its own blocks through a private ring of
-// shared memory with 1-D bulk async copies (payload + 64 scales + 64 zeros +
-// this block column's x' slice), several blocks ahead of the one it is
-// computing.  A warp computes a whole 64x128 block: codes are turned into
-// exact fp16 (q - z) pairs in registers (magic-number OR, then one HFMA2) and
-// multiplied on the tensor cores with mma.m16n8k16 (fp32 accumulation, one
-// group = 8 MMAs per 16 rows); the group result is scaled by s in fp32.
-// At the end of each block row the 4 warps' partial sums are added in a fixed
-// order.  A block row that is split between CTAs is finished by the last CTA
-// to arrive (a per-row counter), which adds the CTAs' partials in unit order,
+// Work split.  At pack time the blocks are cut into `n_units` row-major runs
+// of about equal estimated cost (bytes moved plus decode work per bit
+// width); each run is one warp's work.  A unit descriptor of 128 bytes holds
+// everything the warp needs to start: its run [t0, t1), the offsets of its
+// first block of every width in the code segments and in the scale/zero
+// arrays, the bit widths of its first 64 blocks, and where the partial sums
+// of its first and last block rows go.  One coalesced load of it is the only
+// dependent fetch before the first payload copy is issued.
+//
+// Each warp streams its non-zero blocks through a private ring of shared
+// memory with 1-D bulk async copies (payload + 64 scales + 64 zeros + the
+// activation slice in the column order of the block's low piece + F),
+// several blocks ahead of the one it computes.  Codes become exact fp16
+// subnormal pairs (q - z) * 2^-24 in registers (an AND or byte permute and
+// one HFMA2 per pair; the high piece of a split code is added in before the
+// multiply) and are multiplied on the tensor cores (mma.m16n8k16, fp32
+// accumulation).  Per block and output row: acc += s * F * c.  Forming
+// q - z per element keeps every product exact, so the fp32 rounding stays
+// relative to sum |x * w_hat| even when most codes equal the zero point.
+//
+// A block row that lies inside one run is written straight to y.  A block
+// row shared by several runs (the first and last row of a run) is finished
+// by the last warp to arrive (a per-row arrival counter): it adds the
+// contributors' partial sums -- a contiguous range of slots -- in run order,
 // so results are deterministic.
 //
-// Every wait is bounded: after ~2 s a wait records MPQ_ERR_TIMEOUT, sets a
-// CTA-wide abort flag and the kernel winds down through the same barriers.
+// Every wait is bounded: after ~2 s it records MPQ_ERR_TIMEOUT and the warp
+// stops computing (its arithmetic is skipped, its bookkeeping still runs).
 #pragma once
 #include "common.cuh"
-#include "k_xprep.cuh"   // XQD_SLICE
+#include "k_xprep.cuh"   // XQD_*
 
 namespace mpq {
 
+constexpr uint64_t DEC_WAIT_NS = 2000000000ull;
+
+// Unit descriptor: 32 words.
+enum DescWord {
+    DW_T0 = 0, DW_T1 = 1, DW_SZ = 2,
+    DW_CODE = 3,           // 3..9: code offset of the run's first block of width 1,2,3,4,5,6,8
+    DW_A_SLOT = 10,        // first block row of the run: first partial slot of the row,
+    DW_A_NC = 11,          //   number of runs that meet the row, this run's index among them
+    DW_A_IDX = 12,
+    DW_B_SLOT = 13,        // last block row of the run: the same three
+    DW_B_NC = 14,
+    DW_B_IDX = 15,
+    DW_BITS = 16,          // 16..31: bit widths of the run's first 64 blocks (bytes)
+    DESC_WORDS = 32
+};
+constexpr int DESC_INLINE_BITS = 64;
+
 struct DecodeParams {
     const uint8_t* codes;
-    const mpq_block* table;
-    const uint32_t* sched;
+    const uint32_t* desc;     // [n_units][32]
+    const uint8_t* bits8;     // [NB*KB] bit width per block (runs longer than 64 blocks)
     const uint16_t* scales;
     const uint16_t* zeros;
     const int32_t* row_perm;
-    const uint8_t* xq;        // k_xprep_decode layout: [KB][M_total][272 B]
+    const uint8_t* xq;        // k_xprep_decode records: [KB][XQD_REC * M_total]
     float* y;                 // [M_total][N]
-    float* partial;           // [2*n_units][64][8]
-    uint32_t* counters;       // [NB]
+    float* partial;           // [slots][Mg][64]
+    uint32_t* counters;       // [NB] arrivals per block row
     uint32_t* err;
     int N, K, NB, KB;
     int M_total;              // tokens in xq / y
@@ -48,347 +76,362 @@ struct DecodeParams {
 
 constexpr int DEC_WARPS = 4;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
-constexpr int DEC_RING = 10752;      // bytes of ring per warp (>= largest stage)
+constexpr int DEC_RING = 12288;      // bytes of ring per warp (>= largest stage)
 constexpr int DEC_SLOTS = 8;         // stages in flight per warp
-constexpr uint32_t DEC_MAGIC = 0x64006400u;   // fp16 1024.0 in both halves
-constexpr uint64_t DEC_WAIT_NS = 2000000000ull;
+constexpr int DEC_MAX_TOKENS = 8;
 
-struct DecSmem {
-    uint8_t ring[DEC_WARPS][DEC_RING];
-    float red[DEC_WARPS][64][8];
-    uint64_t full[DEC_WARPS][DEC_SLOTS];
-    mpq_block tab[DEC_WARPS][2][32];   // per-warp table chunks (current, next)
+struct DecWarp {
+    uint8_t ring[DEC_RING];
+    uint64_t full[DEC_SLOTS];
     uint4 zero16[4];          // zero B fragments for lanes beyond the token count
-    volatile int abort_flag;
-    volatile int last_flag;
+};
+struct DecSmem {
+    DecWarp w[DEC_WARPS];
 };
 
 // 4 CTAs per SM: 4 x (smem + 1 KB reserved) must fit the SM's 228 KB
 static_assert(4 * (sizeof(DecSmem) + 1024) <= 228 * 1024, "decode smem too large for 4 CTAs/SM");
-static_assert(DEC_RING >= 8 * 1024 + 256 + 272 * 8, "ring must hold the largest stage");
+// largest stage: an 8-bit payload
+static_assert(DEC_RING >= 8 * 1024 + 256 + DEC_MAX_TOKENS * (XQD_VAR + XQD_AUX), "ring too small");
 
-__device__ __forceinline__ uint32_t h2c(float lo, float hi) {
-    return h2_bits(__halves2half2(__float2half_rn(lo), __float2half_rn(hi)));
-}
-
-// ---------------------------------------------------------------------------
-// Code extraction.  For one row, one 8-code group i of this lane's 32 columns
-// and j = 0..3, out[j] = fp16 pair (q[8i+j] - z, q[8i+j+4] - z), exact.
-// ---------------------------------------------------------------------------
-
-// p = 4: word i holds codes 8i..8i+7 as nibbles.  c1 = -(1024 + z), c16 = -(64 + z).
-__device__ __forceinline__ void ext4(uint32_t w, uint32_t c1, uint32_t c16, uint32_t (&o)[4]) {
-    const uint32_t k116 = 0x2C002C00u;  // 1/16
-    const uint32_t w8 = w >> 8;
-    o[0] = h2_bits(__hadd2(bits_h2(lop_and_or(w, 0x000F000Fu, DEC_MAGIC)), bits_h2(c1)));
-    o[1] = hfma2_bits(lop_and_or(w, 0x00F000F0u, DEC_MAGIC), k116, c16);
-    o[2] = h2_bits(__hadd2(bits_h2(lop_and_or(w8, 0x000F000Fu, DEC_MAGIC)), bits_h2(c1)));
-    o[3] = hfma2_bits(lop_and_or(w8, 0x00F000F0u, DEC_MAGIC), k116, c16);
-}
-
-// p = 2: bytes 2i, 2i+1 of the lane's 8 bytes hold codes 8i..8i+7.
-// c[j] = -(1024/4^j + z) in both halves.
-__device__ __forceinline__ void ext2(uint32_t v, int sel, const uint32_t (&c)[4], uint32_t (&o)[4]) {
-    const uint32_t P = __byte_perm(v, 0u, sel);
-    o[0] = h2_bits(__hadd2(bits_h2(lop_and_or(P, 0x00030003u, DEC_MAGIC)), bits_h2(c[0])));
-    o[1] = hfma2_bits(lop_and_or(P, 0x000C000Cu, DEC_MAGIC), 0x34003400u, c[1]);  // 1/4
-    o[2] = hfma2_bits(lop_and_or(P, 0x00300030u, DEC_MAGIC), 0x2C002C00u, c[2]);  // 1/16
-    o[3] = hfma2_bits(lop_and_or(P, 0x00C000C0u, DEC_MAGIC), 0x24002400u, c[3]);  // 1/64
-}
-
-// p = 1: byte i of the lane's word holds codes 8i..8i+7 (bit k = code 8i+k).
-// c[j] = (-(1024/2^j + z), -(1024/2^(j+4) + z)).
-__device__ __forceinline__ void ext1(uint32_t u, int sel, const uint32_t (&c)[4], uint32_t (&o)[4]) {
-    const uint32_t P = __byte_perm(u, 0u, sel);
-    // low half scaled by 2^-j, high half by 2^-(j+4)
-    o[0] = hfma2_bits(lop_and_or(P, 0x00100001u, DEC_MAGIC), 0x2C003C00u, c[0]);
-    o[1] = hfma2_bits(lop_and_or(P, 0x00200002u, DEC_MAGIC), 0x28003800u, c[1]);
-    o[2] = hfma2_bits(lop_and_or(P, 0x00400004u, DEC_MAGIC), 0x24003400u, c[2]);
-    o[3] = hfma2_bits(lop_and_or(P, 0x00800008u, DEC_MAGIC), 0x20003000u, c[3]);
-}
-
-// p = 8: words 2i and 2i+1 hold codes 8i..8i+3 and 8i+4..8i+7 as bytes.
-// c1 = -(1024 + z).
-__device__ __forceinline__ void ext8(uint32_t xa, uint32_t xb, uint32_t c1, uint32_t (&o)[4]) {
-    const uint32_t T0 = __byte_perm(xa, xb, 0x5140);
-    const uint32_t T1 = __byte_perm(xa, xb, 0x7362);
-    o[0] = h2_bits(__hadd2(bits_h2(__byte_perm(T0, 0x64646464u, 0x4140)), bits_h2(c1)));
-    o[1] = h2_bits(__hadd2(bits_h2(__byte_perm(T0, 0x64646464u, 0x4342)), bits_h2(c1)));
-    o[2] = h2_bits(__hadd2(bits_h2(__byte_perm(T1, 0x64646464u, 0x4140)), bits_h2(c1)));
-    o[3] = h2_bits(__hadd2(bits_h2(__byte_perm(T1, 0x64646464u, 0x4342)), bits_h2(c1)));
-}
-
-// High piece of a split code, already multiplied by 2^w (w = low width):
-// the exact values 2^w * hi, no zero point.  Magic-number pairs carry
-// multipliers m (low half) / m' (high half); an HFMA2 with scale 2^w/m and
-// offset -1024*2^w/m removes the magic.  The constants are fp16 bit patterns
-// (low half in bits 0-15).
-// p = 1: m = 2^j, m' = 2^(j+4).
-template <int W>
-__device__ __forceinline__ void ext1_hi(uint32_t u, int sel, uint32_t (&o)[4]) {
-    const uint32_t P = __byte_perm(u, 0u, sel);
-    // W = 2: scale (4/2^j, 4/2^(j+4)); W = 4: scale (16/2^j, 16/2^(j+4))
-    constexpr uint32_t sc2[4] = {0x34004400u, 0x30004000u, 0x2C003C00u, 0x28003800u};
-    constexpr uint32_t of2[4] = {0xDC00EC00u, 0xD800E800u, 0xD400E400u, 0xD000E000u};
-    constexpr uint32_t sc4[4] = {0x3C004C00u, 0x38004800u, 0x34004400u, 0x30004000u};
-    constexpr uint32_t of4[4] = {0xE400F400u, 0xE000F000u, 0xDC00EC00u, 0xD800E800u};
-    const uint32_t msk[4] = {0x00100001u, 0x00200002u, 0x00400004u, 0x00800008u};
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        o[j] = hfma2_bits(lop_and_or(P, msk[j], DEC_MAGIC), W == 2 ? sc2[j] : sc4[j],
-                          W == 2 ? of2[j] : of4[j]);
-}
-// p = 2 (w = 4): m = m' = 4^j: scale 16/4^j, offset -16384/4^j.
-__device__ __forceinline__ void ext2_hi(uint32_t v, int sel, uint32_t (&o)[4]) {
-    const uint32_t P = __byte_perm(v, 0u, sel);
-    constexpr uint32_t sc[4] = {0x4C004C00u, 0x44004400u, 0x3C003C00u, 0x34003400u};
-    constexpr uint32_t of[4] = {0xF400F400u, 0xEC00EC00u, 0xE400E400u, 0xDC00DC00u};
-    const uint32_t msk[4] = {0x00030003u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o[j] = hfma2_bits(lop_and_or(P, msk[j], DEC_MAGIC), sc[j], of[j]);
-}
-
-// Zero-point constants for a row with zero point z (an fp16 integer).
-__device__ __forceinline__ uint32_t zc(float base, float z) { return h2c(-(base + z), -(base + z)); }
-
-// The same constants from z as (z, z) fp16 pair bits: -(base + z) = z*(-1) - base,
-// exact in fp16 (base + z <= 1279).
-__device__ __forceinline__ uint32_t zc2(uint32_t z2, uint32_t neg_base2) {
-    return hfma2_bits(z2, 0xBC00BC00u, neg_base2);
-}
-
-// Low-piece zero-point constants for a row (see the ext* functions).
-template <int P0>
-__device__ __forceinline__ void zero_consts(uint32_t z2, uint32_t (&k)[4]) {
-    if (P0 == 4) {
-        k[0] = zc2(z2, 0xE400E400u);        // -(1024 + z)
-        k[1] = zc2(z2, 0xD400D400u);        // -(64 + z)
-    } else if (P0 == 8) {
-        k[0] = zc2(z2, 0xE400E400u);
-    } else if (P0 == 2) {
-        k[0] = zc2(z2, 0xE400E400u);        // -(1024 + z)
-        k[1] = zc2(z2, 0xDC00DC00u);        // -(256 + z)
-        k[2] = zc2(z2, 0xD400D400u);        // -(64 + z)
-        k[3] = zc2(z2, 0xCC00CC00u);        // -(16 + z)
-    } else {
-        k[0] = zc2(z2, 0xD400E400u);        // (-(1024 + z), -(64 + z))
-        k[1] = zc2(z2, 0xD000E000u);        // (-(512 + z),  -(32 + z))
-        k[2] = zc2(z2, 0xCC00DC00u);        // (-(256 + z),  -(16 + z))
-        k[3] = zc2(z2, 0xC800D800u);        // (-(128 + z),  -(8 + z))
-    }
-}
+__host__ __device__ constexpr int lo_width(int b) { return (b == 3) ? 2 : (b == 5 || b == 6) ? 4 : b; }
+__host__ __device__ constexpr int hi_width(int b) { return (b == 3 || b == 5) ? 1 : (b == 6) ? 2 : 0; }
+__host__ __device__ constexpr int variant_of(int p) { return p == 1 ? 0 : p == 2 ? 1 : p == 4 ? 2 : 3; }
+// index of width b in the descriptor's code offsets (1,2,3,4,5,6,8 -> 0..6)
+__host__ __device__ constexpr int width_index(int b) { return b == 8 ? 6 : b - 1; }
 
 // ---------------------------------------------------------------------------
-// One 64x128 block of width B.  The lane owns rows 16rt+g and 16rt+g+8 of the
-// four 16-row tiles rt and, in each row, the 32 columns of quad lane t.
-// acc[rt][*] += s_row * 2^-e_tok * sum_k x * (q - z)  (fp32, C-fragment order).
-// The loop over the 4 code groups i is rolled (small code: all 7 widths stay
-// in the instruction cache); inside it the 4 row tiles are independent mma
-// chains.  stage: payload (1024*B) | scales (64 fp16) | zeros (64 fp16) | x'.
+// Code extraction.  For one row and the lane's 32 columns, a[pi] becomes the
+// fp16 pair ((q_a - z) * 2^-24, (q_b - z) * 2^-24) of pair pi (column order
+// of k_xprep.cuh) -- exact subnormals.  An AND (or byte permute) leaves a
+// code at bit `pos` of each half, i.e. the value q * 2^(pos-24); one HFMA2
+// with 2^-pos and zc = -z * 2^-24 gives (q - z) * 2^-24.  A split code adds
+// its high piece the same way, times 2^(low width), before the mma.
 // ---------------------------------------------------------------------------
-template <int B>
-__device__ __forceinline__ void block_mma(const uint8_t* stage, const uint8_t* xs_lane,
-                                          float f0, float f1, float (&acc)[4][4], int g, int t) {
-    const uint16_t* sc = reinterpret_cast<const uint16_t*>(stage + 1024 * B);
-    const uint16_t* zr = sc + 64;
-    constexpr int P0 = (B == 3) ? 2 : (B == 5 || B == 6) ? 4 : B;   // low piece width
-    constexpr int P1 = (B == 3 || B == 5) ? 1 : (B == 6) ? 2 : 0;   // high piece width
-    constexpr int NK = (P0 == 1 || P0 == 2) ? 4 : (P0 == 4 ? 2 : 1);
-    // per-row zero-point constants; rows 16rt+g (index 2rt) and +8 (2rt+1)
-    uint32_t k[8][NK];
+__device__ __forceinline__ constexpr uint32_t h2pow(int k) {      // (2^k, 2^k) fp16 bits
+    return (uint32_t)((15 + k) << 10) * 0x10001u;
+}
+__device__ __forceinline__ uint32_t hadd2_bits(uint32_t a, uint32_t b) {
+    return h2_bits(__hadd2(bits_h2(a), bits_h2(b)));
+}
+
+template <int P>
+__device__ __forceinline__ void extract_lo(const uint32_t (&w)[P], uint32_t zc, uint32_t (&a)[16]) {
+    if (P == 1) {
+        const uint32_t u = w[0], v = w[0] >> 8;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const int r = 8 * q + g;   // q = 2rt + h  ->  row 16rt + 8h + g
-        uint32_t kk[4];
-        zero_consts<P0>(__byte_perm((uint32_t)zr[r], 0u, 0x1010), kk);
+        for (int s = 0; s < 8; ++s) {
+            a[s] = hfma2_bits(u & (0x00010001u << s), h2pow(-s), zc);
+            a[8 + s] = hfma2_bits(v & (0x00010001u << s), h2pow(-s), zc);
+        }
+    } else if (P == 2) {
 #pragma unroll
-        for (int c = 0; c < NK; ++c) k[q][c] = kk[c];
-    }
-    float cg[4][4];
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t u = w[i], v = w[i] >> 8;
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) cg[rt][c] = 0.f;
-    const uint8_t* lo_base = stage + t * 4 * P0;
-    const uint8_t* hi_base = stage + 64 * 16 * P0 + t * 4 * P1;
-#pragma unroll 1
-    for (int i = 0; i < 4; ++i) {
-        const uint4 bv = *reinterpret_cast<const uint4*>(xs_lane + 16 * i);   // B regs 4i..4i+3
-        const int sel2 = (i & 1) ? 0x4342 : 0x4140;
-        const int sel1 = i | (4 << 4) | (i << 8) | (4 << 12);
-#pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
-            uint32_t a[2][4];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = 16 * rt + 8 * h + g;
-                const uint32_t* kq = k[2 * rt + h];
-                const uint8_t* rowp = lo_base + r * 16 * P0;
-                if (P0 == 4) {
-                    const uint32_t w = reinterpret_cast<const uint32_t*>(rowp)[i];
-                    ext4(w, kq[0], kq[1], a[h]);
-                } else if (P0 == 8) {
-                    const uint2 w = reinterpret_cast<const uint2*>(rowp)[i];
-                    ext8(w.x, w.y, kq[0], a[h]);
-                } else if (P0 == 2) {
-                    const uint32_t w = reinterpret_cast<const uint32_t*>(rowp)[i >> 1];
-                    uint32_t kk[4] = {kq[0], kq[1], kq[2], kq[3]};
-                    ext2(w, sel2, kk, a[h]);
-                } else {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(rowp);
-                    uint32_t kk[4] = {kq[0], kq[1], kq[2], kq[3]};
-                    ext1(w, sel1, kk, a[h]);
-                }
-                if (P1 > 0) {   // (lo - z) + 2^w * hi, exact small integers
-                    const uint8_t* hrow = hi_base + r * 16 * P1;
-                    uint32_t hv[4];
-                    if (P1 == 1) ext1_hi<P0>(*reinterpret_cast<const uint32_t*>(hrow), sel1, hv);
-                    else ext2_hi(reinterpret_cast<const uint32_t*>(hrow)[i >> 1], sel2, hv);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) a[h][j] = h2_bits(__hadd2(bits_h2(a[h][j]), bits_h2(hv[j])));
-                }
+            for (int s = 0; s < 4; ++s) {
+                a[8 * i + s] = hfma2_bits(u & (0x00030003u << (2 * s)), h2pow(-2 * s), zc);
+                a[8 * i + 4 + s] = hfma2_bits(v & (0x00030003u << (2 * s)), h2pow(-2 * s), zc);
             }
-            mma_16816(cg[rt], a[0][0], a[1][0], a[0][1], a[1][1], bv.x, bv.y);
-            mma_16816(cg[rt], a[0][2], a[1][2], a[0][3], a[1][3], bv.z, bv.w);
+        }
+    } else if (P == 4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t u = w[i], v = w[i] >> 8;
+            a[4 * i + 0] = hadd2_bits(u & 0x000F000Fu, zc);
+            a[4 * i + 1] = hfma2_bits(u & 0x00F000F0u, h2pow(-4), zc);
+            a[4 * i + 2] = hadd2_bits(v & 0x000F000Fu, zc);
+            a[4 * i + 3] = hfma2_bits(v & 0x00F000F0u, h2pow(-4), zc);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a[2 * i + 0] = hadd2_bits(__byte_perm(w[i], 0u, 0x4240), zc);
+            a[2 * i + 1] = hadd2_bits(__byte_perm(w[i], 0u, 0x4341), zc);
         }
     }
+}
+
+// High piece of a split code added onto the low pairs: a[pi] += 2^w * hi.
+// B = 3: low 2-bit, high 1-bit (w = 2); B = 5: 4 + 1 (w = 4); B = 6: 4 + 2.
+template <int B>
+__device__ __forceinline__ void add_hi(const uint32_t (&h)[B == 6 ? 2 : 1], uint32_t (&a)[16]) {
+    if (B == 3) {
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-        const float s0 = __half2float(__ushort_as_half(sc[16 * rt + g]));
-        const float s1 = __half2float(__ushort_as_half(sc[16 * rt + 8 + g]));
-        acc[rt][0] = fmaf(s0 * f0, cg[rt][0], acc[rt][0]);
-        acc[rt][1] = fmaf(s0 * f1, cg[rt][1], acc[rt][1]);
-        acc[rt][2] = fmaf(s1 * f0, cg[rt][2], acc[rt][2]);
-        acc[rt][3] = fmaf(s1 * f1, cg[rt][3], acc[rt][3]);
+        for (int i = 0; i < 2; ++i) {
+            // bytes 2i, 2i+1 hold the high bits of columns 16i..16i+7, 16i+8..16i+15
+            const uint32_t pb = __byte_perm(h[0], 0u, (2 * i) | (4 << 4) | ((2 * i + 1) << 8) | (4 << 12));
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                a[8 * i + s] = hfma2_bits(pb & (0x00010001u << s), h2pow(2 - s), a[8 * i + s]);
+                a[8 * i + 4 + s] = hfma2_bits(pb & (0x00010001u << (4 + s)), h2pow(-2 - s), a[8 * i + 4 + s]);
+            }
+        }
+    } else if (B == 5) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // byte i holds the high bits of columns 8i..8i+7, in both halves
+            const uint32_t pb = __byte_perm(h[0], 0u, i | (4 << 4) | (i << 8) | (4 << 12));
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                // column 8i+r at bit r (low half), 8i+r+4 at bit r+4 (high half)
+                const uint32_t m = (uint32_t)((15 + 4 - r) << 10) | ((uint32_t)((15 - r) << 10) << 16);
+                a[4 * i + r] = hfma2_bits(pb & ((1u << r) | (1u << (20 + r))), m, a[4 * i + r]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int b0 = 2 * (i & 1);
+            const uint32_t pb = __byte_perm(h[i >> 1], 0u, b0 | (4 << 4) | ((b0 + 1) << 8) | (4 << 12));
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                a[4 * i + r] = hfma2_bits(pb & (0x00030003u << (2 * r)), h2pow(4 - 2 * r), a[4 * i + r]);
+        }
     }
 }
 
+template <int P>
+__device__ __forceinline__ void load_words(const uint8_t* p, uint32_t (&w)[P]) {
+    if (P == 1) {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else if (P == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = v.x; w[1] = v.y;
+    } else if (P == 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+        const uint4 v0 = reinterpret_cast<const uint4*>(p)[0];
+        const uint4 v1 = reinterpret_cast<const uint4*>(p)[1];
+        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+        w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    }
+}
+
+// One row's 16 pairs for width B (stage = payload; lane offset t).
+template <int B>
+__device__ __forceinline__ void row_pairs(const uint8_t* stage, int r, int t, uint32_t zc,
+                                          uint32_t (&a)[16]) {
+    constexpr int P0 = lo_width(B), P1 = hi_width(B);
+    uint32_t w[P0];
+    load_words<P0>(stage + r * 16 * P0 + t * 4 * P0, w);
+    extract_lo<P0>(w, zc, a);
+    if (P1) {
+        uint32_t h[B == 6 ? 2 : 1];
+        const uint8_t* hp = stage + 64 * 16 * P0 + r * 16 * P1 + t * 4 * P1;
+        if (B == 6) {
+            const uint2 v = *reinterpret_cast<const uint2*>(hp);
+            h[0] = v.x; h[B == 6 ? 1 : 0] = v.y;
+        } else {
+            h[0] = *reinterpret_cast<const uint32_t*>(hp);
+        }
+        add_hi<B>(h, a);
+    }
+}
+
+// cg[rt][*] = 2^-24 * sum over the block's 128 columns of (q - z) * x'
+// (C-fragment order: rows 16rt+g, 16rt+g+8 x tokens 2t, 2t+1).
+template <int B>
+__device__ __forceinline__ void block_mma(const uint8_t* stage, const uint32_t (&b)[16],
+                                          float (&cg)[4][4], int g, int t) {
+    const uint16_t* zr16 = reinterpret_cast<const uint16_t*>(stage + 1024 * B) + 64;
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt) {
+        const int r0 = 16 * rt + g, r1 = r0 + 8;
+        // zc = -z * 2^-24 in both halves (z is an fp16 integer; 0x8001 = -2^-24)
+        const uint32_t zc0 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)zr16[r0], 0u, 0x1010)),
+                                             bits_h2(0x80018001u)));
+        const uint32_t zc1 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)zr16[r1], 0u, 0x1010)),
+                                             bits_h2(0x80018001u)));
+        uint32_t a0[16], a1[16];
+        row_pairs<B>(stage, r0, t, zc0, a0);
+        row_pairs<B>(stage, r1, t, zc1, a1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_16816(c, a0[2 * ks], a1[2 * ks], a0[2 * ks + 1], a1[2 * ks + 1], b[2 * ks], b[2 * ks + 1]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cg[rt][k] = c[k];
+    }
+}
+
+__device__ __forceinline__ void load_bfrag(const uint8_t* src, uint32_t (&b)[16]) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = s4[i];
+        b[4 * i] = v.x; b[4 * i + 1] = v.y; b[4 * i + 2] = v.z; b[4 * i + 3] = v.w;
+    }
+}
+
+// Stage layout in the ring (all parts 16-byte multiples):
+//   payload 1024*b | scales 128 | zeros 128 | x' variant of the low piece
+//   256*Mg | F 16*Mg
+__device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
+    return 1024u * b + 256u + (XQD_VAR + XQD_AUX) * Mg;
+}
+
 // ---------------------------------------------------------------------------
-// The kernel
+// The kernel.  ONE_TOKEN: the launch has Mg == 1 (only C-fragment column 0
+// carries data, so the per-block epilogue handles half the elements).
 // ---------------------------------------------------------------------------
+template <bool ONE_TOKEN>
 __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int u = blockIdx.x;
-    const int KB = p.KB;
+    DecWarp& W = S.w[warp];
+    const int u = blockIdx.x * DEC_WARPS + warp;
+    const uint32_t KB = (uint32_t)p.KB;
+    const uint32_t lt_mask = (1u << lane) - 1u;
 
-    if (tid == 0) {
-        for (int w = 0; w < DEC_WARPS; ++w)
-            for (int s = 0; s < DEC_SLOTS; ++s) mbar_init(&S.full[w][s], 1);
-        S.abort_flag = 0;
-        for (int q = 0; q < 4; ++q) S.zero16[q] = make_uint4(0u, 0u, 0u, 0u);
+    if (lane == 0) {
+        for (int s = 0; s < DEC_SLOTS; ++s) mbar_init(&W.full[s], 1);
         fence_mbar_init();
     }
-    const uint32_t t0 = p.sched[u], t1 = p.sched[u + 1];
-    __syncthreads();
-
-    const int Mg = p.Mg;
-    const uint32_t xslice = (uint32_t)XQD_SLICE * (uint32_t)Mg;
-    uint8_t* ring = S.ring[warp];
-
-    // ---- per-warp stream state (uniform across the warp) ----
-    // Table chunks of 32 entries, the next one loaded a chunk ahead.  For the
-    // current chunk, `mine` has a bit for every lane whose block is non-zero
-    // and dealt to this warp (the unit's non-zero blocks go round-robin).
-    uint32_t tab_base = t0 & ~31u;
-    uint32_t nz_before = 0;          // non-zero blocks of this unit before the chunk
-    int tb = 0;                      // which of the two chunk buffers is current
-    // each lane copies its entry of the chunk at `base` (zeros outside [t0, t1))
-    auto fetch = [&](uint32_t base, int buf) {
-        const uint32_t tt = base + lane;
-        const bool in = tt >= t0 && tt < t1;
-        cp_async16(&S.tab[warp][buf][lane], p.table + (in ? tt : t0), in ? 16u : 0u);
-        cp_async_commit();
-    };
-    fetch(tab_base, 0);
-    fetch(tab_base + 32, 1);
-    cp_async_wait_all();
+    if (lane < 4) W.zero16[lane] = make_uint4(0u, 0u, 0u, 0u);
     __syncwarp();
-    auto mine_of = [&]() -> uint32_t {
-        const uint32_t bits = S.tab[warp][tb][lane].bits;
-        const uint32_t nzm = __ballot_sync(0xffffffffu, bits != 0u);
-        const uint32_t rank = nz_before + __popc(nzm & ((1u << lane) - 1u));
-        const uint32_t m = __ballot_sync(0xffffffffu, bits != 0u &&
-                                                          (rank & (DEC_WARPS - 1)) == (uint32_t)warp);
-        nz_before += __popc(nzm);
-        return m;
-    };
-    uint32_t mine = mine_of();
+    if (u >= p.n_units) return;
+
+    // ---- the unit descriptor: lane i holds word i ----
+    const uint32_t dw = __ldg(p.desc + (size_t)u * DESC_WORDS + lane);
+    const uint32_t t0 = __shfl_sync(0xffffffffu, dw, DW_T0);
+    const uint32_t t1 = __shfl_sync(0xffffffffu, dw, DW_T1);
+    uint32_t sz_base = __shfl_sync(0xffffffffu, dw, DW_SZ);
+    // lanes DW_CODE..DW_CODE+6 keep the running code offset of their width
+    uint32_t code_run = dw;
+
+    const uint32_t Mg = (uint32_t)p.Mg;
+    const size_t rec_bytes = (size_t)p.M_total * XQD_REC;
+    const uint8_t* xq_tok = p.xq + (size_t)p.m0 * XQD_VAR;     // + kb*rec + v*M*256
+    const uint8_t* xq_aux = p.xq + (size_t)4 * p.M_total * XQD_VAR + (size_t)p.m0 * XQD_AUX;
+
+    // ---- chunk state: lane l describes block t0 + 32*chunk + l ----
+    uint32_t chunk = 0;
+    uint32_t c_bits = 0, c_code = 0, c_sz = 0;
+    uint32_t pending = 0;            // non-zero blocks of the chunk not yet issued
     bool scan_done = false;
+    uint32_t bits_pref = 0;          // prefetched widths of the next chunk (beyond the inline 64)
+
+    bool aborted = false;            // a bounded wait ran out: stop computing
+    auto load_chunk = [&]() {
+        const uint32_t j = 32u * chunk + (uint32_t)lane;
+        const bool in = t0 + j < t1;
+        // widths of the first 64 blocks are inline in the descriptor
+        const uint32_t jw = min(j, (uint32_t)DESC_INLINE_BITS - 1u);
+        const uint32_t word = __shfl_sync(0xffffffffu, dw, DW_BITS + (int)(jw >> 2));
+        uint32_t b = (j < (uint32_t)DESC_INLINE_BITS) ? (word >> (8 * (j & 3))) & 0xFFu : bits_pref;
+        b = in ? b : 0u;
+        // prefetch the next chunk's widths when they are not inline
+        const uint32_t jn = j + 32u;
+        if (jn >= (uint32_t)DESC_INLINE_BITS && t0 + jn < t1) bits_pref = __ldg(p.bits8 + t0 + jn);
+        c_bits = b;
+        // rank among the chunk's blocks of the same width -> code offset
+        const uint32_t same = __match_any_sync(0xffffffffu, b);
+        const uint32_t rank = __popc(same & lt_mask);
+        const uint32_t base = __shfl_sync(0xffffffffu, code_run, DW_CODE + width_index(b == 0 ? 1 : (int)b));
+        c_code = base + rank * 1024u * b;
+        const uint32_t nz = __ballot_sync(0xffffffffu, b != 0u);
+        c_sz = sz_base + 64u * __popc(nz & lt_mask);
+        sz_base += 64u * __popc(nz);
+        pending = nz;
+    };
+    // advance the running code offsets past the chunk (lane DW_CODE + i owns width i)
+    auto advance_codes = [&]() {
+        uint32_t add = 0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) {
+            const uint32_t wb = (i == 6) ? 8u : (uint32_t)(i + 1);
+            const uint32_t cnt = __popc(__ballot_sync(0xffffffffu, c_bits == wb));
+            if (lane == DW_CODE + i) add = cnt * 1024u * wb;
+        }
+        code_run += add;
+    };
+
+    load_chunk();
+    advance_codes();
+
+    // ---- stage queue: entry k lives in lane k % DEC_SLOTS ----
     uint32_t q_head = 0, q_tail = 0;     // consumed / issued stages
-    uint32_t r_head = 0, r_tail = 0;     // ring bytes issued / freed
-    // queue entry k lives in lane k % DEC_SLOTS
+    uint32_t r_head = 0, r_tail = 0;     // ring bytes issued / freed (monotone)
+    uint32_t r_pos = 0;                  // physical ring offset of r_head
     uint32_t qe_t = 0, qe_bits = 0, qe_off = 0, qe_end = 0;
     bool xq_ready = false;               // x' is written by the prologue kernel
 
-    auto issue_xq = [&](uint32_t tt, uint32_t b, uint32_t off, uint32_t slot) {
+    auto issue_x = [&](uint32_t tt, uint32_t b, uint32_t off, uint32_t slot) {
         const uint32_t kb = tt % KB;
-        bulk_g2s(ring + off + 1024u * b + 256u,
-                 p.xq + ((size_t)kb * p.M_total + p.m0) * XQD_SLICE, xslice, &S.full[warp][slot]);
+        uint8_t* dst = W.ring + off + 1024u * b + 256u;
+        const uint8_t* rec = xq_tok + (size_t)kb * rec_bytes;
+        const uint32_t vb = XQD_VAR * Mg;
+        bulk_g2s(dst, rec + (size_t)variant_of(lo_width((int)b)) * p.M_total * XQD_VAR, vb, &W.full[slot]);
+        bulk_g2s(dst + vb, xq_aux + (size_t)kb * rec_bytes, XQD_AUX * Mg, &W.full[slot]);
     };
     auto issue_more = [&]() {
         while (q_tail - q_head < (uint32_t)DEC_SLOTS && !scan_done) {
-            if (mine == 0u) {
-                if (tab_base + 32 >= t1) { scan_done = true; break; }
-                tab_base += 32;
-                cp_async_wait_all();     // the next chunk landed long ago
-                __syncwarp();
-                tb ^= 1;
-                fetch(tab_base + 32, tb ^ 1);   // refill the buffer just retired
-                mine = mine_of();
+            if (aborted) { scan_done = true; break; }
+            if (pending == 0u) {
+                if (t0 + 32u * (chunk + 1) >= t1) { scan_done = true; break; }
+                ++chunk;
+                load_chunk();
+                advance_codes();
                 continue;
             }
-            if (q_head == q_tail) { r_head = 0; r_tail = 0; }   // empty ring: restart at 0
-            const int l = __ffs(mine) - 1;
-            const mpq_block& en = S.tab[warp][tb][l];
-            const uint32_t b = en.bits;
-            const uint32_t size = 1024u * b + 256u + xslice;
-            uint32_t start = r_head;
-            const uint32_t pos = r_head % DEC_RING;
-            if (pos + size > DEC_RING) start = r_head + (DEC_RING - pos);
-            if (start + size - r_tail > DEC_RING) break;   // ring full: compute first
-            const uint32_t coff = en.code_off;
-            const uint32_t szo = en.sz_off;
-            const uint32_t tt = tab_base + l;
+            if (q_head == q_tail) { r_head = 0; r_tail = 0; r_pos = 0; }   // empty ring: restart at 0
+            const int l = __ffs(pending) - 1;
+            const uint32_t b = __shfl_sync(0xffffffffu, c_bits, l);
+            const uint32_t coff = __shfl_sync(0xffffffffu, c_code, l);
+            const uint32_t szo = __shfl_sync(0xffffffffu, c_sz, l);
+            const uint32_t size = stage_bytes(b, Mg);
+            // a stage never wraps: when the ring's tail end is too short, skip to 0
+            const bool skip = r_pos + size > (uint32_t)DEC_RING;
+            const uint32_t start = skip ? r_head + ((uint32_t)DEC_RING - r_pos) : r_head;
+            if (start + size - r_tail > (uint32_t)DEC_RING) break;   // ring full: compute first
+            const uint32_t tt = t0 + 32u * chunk + (uint32_t)l;
             const uint32_t slot = q_tail % DEC_SLOTS;
-            const uint32_t off = start % DEC_RING;
+            const uint32_t off = skip ? 0u : r_pos;
             if (lane == 0) {
                 fence_proxy_async_smem();
-                uint64_t* bar = &S.full[warp][slot];
+                uint64_t* bar = &W.full[slot];
                 mbar_arrive_expect_tx(bar, size);
-                uint8_t* dst = ring + off;
+                uint8_t* dst = W.ring + off;
                 bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
                 bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
                 bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
-                if (xq_ready) issue_xq(tt, b, off, slot);
+                if (xq_ready) issue_x(tt, b, off, slot);
             }
             if (lane == (int)slot) { qe_t = tt; qe_bits = b; qe_off = off; qe_end = start + size; }
             r_head = start + size;
+            r_pos = off + size;
             ++q_tail;
-            mine &= mine - 1u;
+            pending &= pending - 1u;
         }
     };
 
     // Weights do not depend on the prologue kernel: start streaming them, then
     // wait for x' (programmatic dependent launch) and add its copies.
-    if (t0 < t1) issue_more();
+    issue_more();
     pdl_wait();
-    if (t0 >= t1) return;
     xq_ready = true;
     for (uint32_t k = q_head; k < q_tail; ++k) {
         const uint32_t slot = k % DEC_SLOTS;
         const uint32_t kt = __shfl_sync(0xffffffffu, qe_t, slot);
-        const uint32_t kb_ = __shfl_sync(0xffffffffu, qe_bits, slot);
+        const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
         const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
-        if (lane == 0) issue_xq(kt, kb_, ko, slot);
+        if (lane == 0) issue_x(kt, kbits, ko, slot);
     }
 
-    float* red = &S.red[0][0][0];
     const uint32_t nb_first = t0 / KB, nb_last = (t1 - 1) / KB;
     for (uint32_t nb = nb_first; nb <= nb_last; ++nb) {
-        const uint32_t row_end = min(t1, (nb + 1) * (uint32_t)KB);
+        const uint32_t row_end = min(t1, (nb + 1) * KB);
+        // output rows of this lane: 16rt+g (+8); their permuted indices, early
+        int rp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int i = (int)nb * 64 + 8 * q + g;   // q = 2rt + h -> row 16rt + 8h + g
+            rp[q] = p.row_perm ? __ldg(p.row_perm + i) : i;
+        }
         float acc[4][4];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
@@ -400,32 +443,49 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
             if (q_head == q_tail) break;    // nothing left for this warp at all
             const uint32_t slot = q_head % DEC_SLOTS;
             const uint32_t ft = __shfl_sync(0xffffffffu, qe_t, slot);
-            if (ft >= row_end) break;       // next block of mine is in a later row
+            if (ft >= row_end) break;       // the next block is in a later row
             const uint32_t fb = __shfl_sync(0xffffffffu, qe_bits, slot);
             const uint32_t foff = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t fend = __shfl_sync(0xffffffffu, qe_end, slot);
-            bool ok = true;
-            if (!S.abort_flag) ok = mbar_wait_bounded(&S.full[warp][slot], (q_head / DEC_SLOTS) & 1u, DEC_WAIT_NS);
-            if (!ok) {
-                if (lane == 0) { set_error(p.err, MPQ_ERR_TIMEOUT); S.abort_flag = 1; }
+            if (!aborted) {
+                const bool ok = mbar_wait_bounded(&W.full[slot], (q_head / DEC_SLOTS) & 1u, DEC_WAIT_NS);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    aborted = true;
+                    if (lane == 0) set_error(p.err, MPQ_ERR_TIMEOUT);
+                }
             }
-            __syncwarp();
-            if (!S.abort_flag) {
-                const uint8_t* stage = ring + foff;
+            if (!aborted) {
+                const uint8_t* stage = W.ring + foff;
                 const uint8_t* xs = stage + 1024u * fb + 256u;
-                // this lane's B fragments (token g, quad lane t); zeros beyond Mg
-                const uint8_t* xs_lane = (g < Mg) ? xs + g * XQD_SLICE + t * 64 : reinterpret_cast<const uint8_t*>(S.zero16);
-                // 2^-e of the tokens 2t and 2t+1 (the C-fragment columns)
-                const float f0 = (2 * t < Mg) ? *reinterpret_cast<const float*>(xs + (2 * t) * XQD_SLICE + 256) : 0.f;
-                const float f1 = (2 * t + 1 < Mg) ? *reinterpret_cast<const float*>(xs + (2 * t + 1) * XQD_SLICE + 256) : 0.f;
+                const uint8_t* aux = xs + XQD_VAR * Mg;
+                // this lane's B fragments: token g, quad lane t; zeros beyond Mg
+                uint32_t bf[16];
+                load_bfrag((uint32_t)g < Mg ? xs + g * XQD_VAR + t * 64
+                                            : reinterpret_cast<const uint8_t*>(W.zero16), bf);
+                float cg[4][4];
                 switch (fb) {
-                    case 1: block_mma<1>(stage, xs_lane, f0, f1, acc, g, t); break;
-                    case 2: block_mma<2>(stage, xs_lane, f0, f1, acc, g, t); break;
-                    case 3: block_mma<3>(stage, xs_lane, f0, f1, acc, g, t); break;
-                    case 4: block_mma<4>(stage, xs_lane, f0, f1, acc, g, t); break;
-                    case 5: block_mma<5>(stage, xs_lane, f0, f1, acc, g, t); break;
-                    case 6: block_mma<6>(stage, xs_lane, f0, f1, acc, g, t); break;
-                    default: block_mma<8>(stage, xs_lane, f0, f1, acc, g, t); break;
+                    case 1: block_mma<1>(stage, bf, cg, g, t); break;
+                    case 2: block_mma<2>(stage, bf, cg, g, t); break;
+                    case 3: block_mma<3>(stage, bf, cg, g, t); break;
+                    case 4: block_mma<4>(stage, bf, cg, g, t); break;
+                    case 5: block_mma<5>(stage, bf, cg, g, t); break;
+                    case 6: block_mma<6>(stage, bf, cg, g, t); break;
+                    default: block_mma<8>(stage, bf, cg, g, t); break;
+                }
+                // epilogue: acc += s * F * cg per row and token
+                const uint16_t* sc16 = reinterpret_cast<const uint16_t*>(stage + 1024u * fb);
+                const float Fa = (2u * t < Mg) ? *reinterpret_cast<const float*>(aux + (2 * t) * XQD_AUX) : 0.f;
+                const float Fb = (!ONE_TOKEN && 2u * t + 1u < Mg)
+                                     ? *reinterpret_cast<const float*>(aux + (2 * t + 1) * XQD_AUX) : 0.f;
+#pragma unroll
+                for (int rt = 0; rt < 4; ++rt) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float sr = __half2float(__ushort_as_half(sc16[16 * rt + 8 * h + g]));
+                        // F * cg is the block's sum at the activations' own scale
+                        acc[rt][2 * h] = fmaf(sr, Fa * cg[rt][2 * h], acc[rt][2 * h]);
+                        if (!ONE_TOKEN) acc[rt][2 * h + 1] = fmaf(sr, Fb * cg[rt][2 * h + 1], acc[rt][2 * h + 1]);
+                    }
                 }
             }
             __syncwarp();
@@ -433,76 +493,89 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
             r_tail = fend;
         }
 
-        // ---- end of block row nb: add the 4 warps' partials in a fixed order ----
-#pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
-            float* rw = red + ((size_t)warp * 64 + 16 * rt + g) * 8;
-            *reinterpret_cast<float2*>(rw + 2 * t) = make_float2(acc[rt][0], acc[rt][1]);
-            *reinterpret_cast<float2*>(rw + 64 + 2 * t) = make_float2(acc[rt][2], acc[rt][3]);
+        // ---- end of block row nb ----
+        uint32_t slot_base = 0, nc = 1, idx = 0;
+        if (nb == nb_first) {
+            slot_base = __shfl_sync(0xffffffffu, dw, DW_A_SLOT);
+            nc = __shfl_sync(0xffffffffu, dw, DW_A_NC);
+            idx = __shfl_sync(0xffffffffu, dw, DW_A_IDX);
+        } else if (nb == nb_last) {
+            slot_base = __shfl_sync(0xffffffffu, dw, DW_B_SLOT);
+            nc = __shfl_sync(0xffffffffu, dw, DW_B_NC);
+            idx = __shfl_sync(0xffffffffu, dw, DW_B_IDX);
         }
-        named_bar_sync(1, DEC_THREADS);
-        const bool complete = (nb * (uint32_t)KB >= t0) && ((nb + 1) * (uint32_t)KB <= t1);
-        float sums[4];
-        int rows[4], toks[4];
+        // tokens 2t, 2t+1 of rows 16rt+g, 16rt+g+8
+        const int tok_a = 2 * t, tok_b = 2 * t + 1;
+        const bool wa = (uint32_t)tok_a < Mg, wb = !ONE_TOKEN && (uint32_t)tok_b < Mg;
+        if (nc == 1u) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int idx = lane + 32 * q;           // 16 rows x 8 tokens per warp
-            rows[q] = 16 * warp + (idx >> 3);
-            toks[q] = idx & 7;
-            const size_t o = (size_t)rows[q] * 8 + toks[q];
-            sums[q] = ((red[o] + red[64 * 8 + o]) + red[2 * 64 * 8 + o]) + red[3 * 64 * 8 + o];
+            for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int n = rp[2 * rt + h];
+                    if (wa) p.y[(size_t)(p.m0 + tok_a) * p.N + n] = acc[rt][2 * h];
+                    if (wb) p.y[(size_t)(p.m0 + tok_b) * p.N + n] = acc[rt][2 * h + 1];
+                }
+            continue;
         }
-        if (complete) {
+        // shared row: deposit this run's partial sums, then count the arrival
+        {
+            float* part = p.partial + (size_t)(slot_base + idx) * Mg * 64;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (toks[q] < Mg) {
-                    const int i = (int)nb * 64 + rows[q];
-                    const int n = p.row_perm ? p.row_perm[i] : i;
-                    p.y[(size_t)(p.m0 + toks[q]) * p.N + n] = sums[q];
+            for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = 16 * rt + 8 * h + g;
+                    if (wa) part[tok_a * 64 + r] = acc[rt][2 * h];
+                    if (wb) part[tok_b * 64 + r] = acc[rt][2 * h + 1];
                 }
-            }
-        } else {
-            const uint32_t first_row = t0 / KB;
-            const uint32_t slot_id = 2u * (uint32_t)u + (nb == first_row ? 0u : 1u);
-            float* part = p.partial + (size_t)slot_id * 64 * 8;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) part[rows[q] * 8 + toks[q]] = sums[q];
-            // the CTA barrier orders every thread's partial before thread 0's
-            // release; the acquire side is thread 0's atomic + the barrier
-            named_bar_sync(1, DEC_THREADS);
-            if (tid == 0) {
-                const uint32_t lo = max(t0, nb * (uint32_t)KB);
-                const uint32_t cnt = row_end - lo;
-                const uint32_t old = atomic_add_acq_rel_gpu(&p.counters[nb], cnt);
-                S.last_flag = (old + cnt == (uint32_t)KB);
-            }
-            named_bar_sync(1, DEC_THREADS);
-            if (S.last_flag) {
-                // contributors: the units whose runs meet block row nb
-                uint32_t c_first = (uint32_t)u, c_last = (uint32_t)u;
-                while (p.sched[c_first] > nb * (uint32_t)KB) --c_first;
-                while (p.sched[c_last + 1] < (nb + 1) * (uint32_t)KB) ++c_last;
-                float tot[4] = {0.f, 0.f, 0.f, 0.f};
-                for (uint32_t c = c_first; c <= c_last; ++c) {
-                    const uint32_t cs = p.sched[c], ce = p.sched[c + 1];
-                    if (cs >= ce) continue;
-                    const uint32_t sid = 2u * c + ((cs / KB) == nb ? 0u : 1u);
-                    const float* pc = p.partial + (size_t)sid * 64 * 8;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) tot[q] += __ldcg(pc + rows[q] * 8 + toks[q]);
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (toks[q] < Mg) {
-                        const int i = (int)nb * 64 + rows[q];
-                        const int n = p.row_perm ? p.row_perm[i] : i;
-                        p.y[(size_t)(p.m0 + toks[q]) * p.N + n] = tot[q];
-                    }
-                }
-                if (tid == 0) p.counters[nb] = 0u;   // ready for the next launch
-            }
         }
-        named_bar_sync(1, DEC_THREADS);   // red[] is reused by the next row
+        // __syncwarp orders every lane's partial before lane 0's release; the
+        // acquire side is lane 0's atomic + __syncwarp, then L2 (.cg) loads
+        __syncwarp();
+        uint32_t last = 0;
+        if (lane == 0) last = (atomic_add_acq_rel_gpu(&p.counters[nb], 1u) + 1u == nc) ? 1u : 0u;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        __syncwarp();
+        if (!last) continue;
+        float tot[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tot[a][c] = 0.f;
+#pragma unroll 4
+        for (uint32_t c = 0; c < nc; ++c) {
+            // the slots of the row's runs, in run order (deterministic sum)
+            const float* pc = p.partial + (size_t)(slot_base + c) * Mg * 64;
+            float v[4][4];
+#pragma unroll
+            for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = 16 * rt + 8 * h + g;
+                    v[rt][2 * h] = wa ? __ldcg(pc + tok_a * 64 + r) : 0.f;
+                    v[rt][2 * h + 1] = wb ? __ldcg(pc + tok_b * 64 + r) : 0.f;
+                }
+            if (c == idx) {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) v[a][cc] = acc[a][cc];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) tot[a][cc] += v[a][cc];
+        }
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int n = rp[2 * rt + h];
+                if (wa) p.y[(size_t)(p.m0 + tok_a) * p.N + n] = tot[rt][2 * h];
+                if (wb) p.y[(size_t)(p.m0 + tok_b) * p.N + n] = tot[rt][2 * h + 1];
+            }
+        if (lane == 0) p.counters[nb] = 0u;   // ready for the next launch
     }
 }
 

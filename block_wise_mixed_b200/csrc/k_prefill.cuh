@@ -32,7 +32,8 @@
 #include <cuda.h>
 
 #include "common.cuh"
-#include "k_decode.cuh"   // code extraction helpers (ext1/2/4/8, *_hi)
+#include "dequant_magic.cuh"
+#include "k_decode.cuh"       // DEC_WAIT_NS
 
 namespace mpq {
 

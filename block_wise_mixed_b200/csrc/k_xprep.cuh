@@ -19,13 +19,8 @@
 //               which the tensor-core kernel's dequantization emits weights.
 // Block 0 also clears the workspace error word.
 //
-// k_xprep_decode (below) is the small-batch variant: one warp per (block
-// column kb, token m) and no row-wide reduction.  Each 128-column slice gets
-// its own power of two 2^e (from the slice's largest magnitude), stored with
-// the slice; the decode kernel folds 2^-e into its per-group fp32 scale.
-// Layout [KB][M][272 bytes]: 4 quad lanes x 16 half2 in the mma B-fragment
-// order of XP_DECODE, then the fp32 factor 2^-e and 12 bytes of padding.
-// It also clears the decode kernel's per-block-row counters.
+// k_xprep_decode (below) is the small-batch variant; its layout is described
+// there.
 #pragma once
 #include "common.cuh"
 
@@ -116,18 +111,65 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
     }
 }
 
-constexpr int XQD_SLICE = 272;   // bytes per (kb, token) slice
+// ---------------------------------------------------------------------------
+// Small-batch activation records (k_xprep_decode).
+//
+// The decode kernel turns a pair of packed codes into the fp16 pair
+// ((q_a - z) * 2^-24, (q_b - z) * 2^-24) -- exact subnormals -- with one AND
+// (or byte permute) and one HFMA2 per pair.  Which two columns share a pair
+// follows from where a p-bit piece puts its codes in a 32-bit word (the two
+// 16-bit halves), so each piece width p = 1, 2, 4, 8 pairs the columns in its
+// own order, and the activation slice is stored once per order ("variant").
+// For quad lane t of the mma, pair index pi (0..15) of a row's 32 columns
+// 32t..32t+31 holds the columns (colA, colB):
+//   p = 1: cols (s + 8*(pi/8), s + 8*(pi/8) + 16),  s = pi % 8
+//   p = 2: cols (16i + 4h + s, 16i + 4h + s + 8),   i = pi/8, h = (pi/4)%2, s = pi%4
+//   p = 4: cols (8i + r, 8i + r + 4),               i = pi/4, r = pi % 4
+//   p = 8: cols (4i + r, 4i + r + 2),               i = pi/2, r = pi % 2
+// and register pi of the mma B fragment is (x'[colA], x'[colB]).
+//
+// Each 128-column slice (block column kb) of token m is scaled by its own
+// power of two 2^e (amax * 2^e in [2^14, 2^15), e >= -103), so that bf16
+// values are exact in fp16.  The tensor cores then accumulate
+// c_r = 2^-24 * sum_j (q_j - z_r) x'_j, and the block adds s_r * F * c_r to
+// output row r, with F = 2^(24 - e).
+//
+// Record of block column kb (XQD_REC * M bytes, 16-byte aligned):
+//   [v = 0..3 (p = 1, 2, 4, 8)][m][t = 0..3][pi = 0..15] half2   (4*256*M B)
+//   [m] float4 (F, 0, 0, 0)                                       (16*M B)
+// so one variant of a token group is one contiguous run of 256*Mg bytes.
+// Block 0 also clears the workspace error word and the decode kernel's
+// per-block-row counters.
+// ---------------------------------------------------------------------------
+constexpr int XQD_VAR = 256;                 // one variant of one token
+constexpr int XQD_AUX = 16;                  // F of one token (padded)
+constexpr int XQD_REC = 4 * XQD_VAR + XQD_AUX;
+
+__device__ __forceinline__ void xqd_pair_cols(int v, int pi, int& ca, int& cb) {
+    if (v == 0) {
+        ca = (pi & 7) + 8 * (pi >> 3); cb = ca + 16;
+    } else if (v == 1) {
+        ca = 16 * (pi >> 3) + 4 * ((pi >> 2) & 1) + (pi & 3); cb = ca + 8;
+    } else if (v == 2) {
+        ca = 8 * (pi >> 2) + (pi & 3); cb = ca + 4;
+    } else {
+        ca = 4 * (pi >> 1) + (pi & 1); cb = ca + 2;
+    }
+}
+
+constexpr int XPREP_DEC_WARPS = XPREP_THREADS / 32;
 
 __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
     pdl_launch_dependents();
-    const int tid = threadIdx.x, lane = tid & 31;
+    __shared__ float xs[XPREP_DEC_WARPS][64];   // 128 fp16 per warp
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int KB = p.K / 128;
     if (blockIdx.x == 0) {
         if (tid == 0 && p.err) *p.err = 0u;
         if (p.counters)
             for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
     }
-    const int item = blockIdx.x * (XPREP_THREADS / 32) + (tid >> 5);   // = kb * M + m
+    const int item = blockIdx.x * XPREP_DEC_WARPS + warp;   // = kb * M + m
     if (item >= KB * p.M) return;
     const int kb = item / p.M, m = item % p.M;
     const uint16_t* xr = p.x + (size_t)m * p.K;
@@ -151,7 +193,7 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
 #pragma unroll
     for (int e4 = 0; e4 < 4; ++e4) {
         const float a = fabsf(v[e4]);
-        amax = (a > amax || a != a) ? a : amax;
+        amax = (a > amax || a != a) ? a : amax;   // NaN-propagating max
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -159,25 +201,29 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
         amax = (o > amax || o != o) ? o : amax;
     }
     int e = 0;
-    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -126), 126);
-    // pair (8i+j, 8i+j+4): columns 8i..8i+3 sit in lane 2i', 8i+4..8i+7 in lane 2i'+1
-    float w[4];
+    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -103), 126);
+    // x' = fp16(x * 2^e) (exact for bf16 inputs in range)
+    __half* xw = reinterpret_cast<__half*>(xs[warp]);
 #pragma unroll
-    for (int e4 = 0; e4 < 4; ++e4) w[e4] = __shfl_down_sync(0xffffffffu, v[e4], 1);
-    uint8_t* slice = reinterpret_cast<uint8_t*>(p.xq) + (size_t)item * XQD_SLICE;
-    if ((lane & 1) == 0) {
-        // this lane's 8 columns are 8*(lane/2) .. +7 of the slice: quad lane
-        // t = lane/8, group i = (lane/2) % 4, registers 4i .. 4i+3
-        uint4 out;
-        uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+    for (int e4 = 0; e4 < 4; ++e4) xw[4 * lane + e4] = __float2half_rn(ldexpf(v[e4], e));
+    __syncwarp();
+    // lane -> variant vv = lane / 8, quad lane tq = (lane / 2) % 4, pairs 8*(lane % 2) .. +7
+    const int vv = lane >> 3, tq = (lane >> 1) & 3, pi0 = 8 * (lane & 1);
+    uint32_t o[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            o[j] = h2_bits(__halves2half2(__float2half_rn(ldexpf(v[j], e)), __float2half_rn(ldexpf(w[j], e))));
-        *reinterpret_cast<uint4*>(slice + (lane >> 1) * 16) = out;
+    for (int i = 0; i < 8; ++i) {
+        int ca, cb;
+        xqd_pair_cols(vv, pi0 + i, ca, cb);
+        o[i] = h2_bits(__halves2half2(xw[32 * tq + ca], xw[32 * tq + cb]));
     }
-    if (lane == 0) {
-        *reinterpret_cast<float4*>(slice + 256) = make_float4(ldexpf(1.f, -e), 0.f, 0.f, 0.f);
-    }
+    uint8_t* rec = reinterpret_cast<uint8_t*>(p.xq) + (size_t)kb * p.M * XQD_REC;
+    uint4* dst = reinterpret_cast<uint4*>(rec + (size_t)vv * p.M * XQD_VAR + (size_t)m * XQD_VAR +
+                                          tq * 64 + pi0 * 4);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    if (lane == 0)
+        *reinterpret_cast<float4*>(rec + (size_t)4 * p.M * XQD_VAR + (size_t)m * XQD_AUX) =
+            make_float4(ldexpf(1.f, 24 - e), 0.f, 0.f, 0.f);
 }
 
 }  // namespace mpq

@@ -22,9 +22,9 @@ using namespace mpq;
 
 namespace {
 
-constexpr int kMaxUnits = 592;          // 4 decode CTAs on each of 148 SMs
-constexpr uint64_t kMinUnitBits = 8;    // >= 8 KiB of codes per decode unit
-constexpr int kMaxDecodeTokens = 8;     // tokens per decode launch
+constexpr int kMaxUnits = 148 * 16;    // one run per resident decode warp (16 per SM)
+constexpr uint64_t kMinUnitCost = 4096; // cost units (bytes) per run, at least
+constexpr int kMaxDecodeTokens = DEC_MAX_TOKENS;   // tokens per decode launch
 constexpr int kDecodeMaxM = 16;         // larger batches take the tensor-core kernel
 constexpr int kPackRowsPerCta = 16;
 
@@ -32,7 +32,22 @@ inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
 inline bool bits_ok(int b) { return b == 0 || b == 1 || b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8; }
 
+// Estimated cost of one block for the decode schedule, in bytes: what it
+// streams (payload, scales/zeros, one activation variant) plus a stand-in
+// for its decode work (code extraction and tensor-core passes).  Split
+// widths (3, 5, 6) make two passes.  Zero-bit blocks only cost bookkeeping.
+inline uint64_t block_cost(int b) {
+    static const uint32_t work[9] = {0, 2048, 2048, 4096, 2304, 4352, 4352, 0, 2560};
+    return b == 0 ? 32u : 1024u * (uint64_t)b + 256u + 272u + work[b];
+}
+
+inline uint64_t sched_words_of(int64_t n_units, int64_t T) {
+    return (uint64_t)n_units * DESC_WORDS + (uint64_t)(T + 3) / 4;
+}
+
 // Layout of the plan for (N, K, bits) -- the same arithmetic as mpq_plan.
+// sched (optional) receives the decode schedule: n_units descriptors of
+// DESC_WORDS words (see k_decode.cuh), then one byte per block (its width).
 mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
                      std::vector<mpq_block>* table, std::vector<uint32_t>* sched) {
     if (N <= 0 || K <= 0 || N % 64 != 0 || K % 128 != 0) return MPQ_ERR_SHAPE;
@@ -58,16 +73,35 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
     for (int64_t t = 0; t < T; ++t) total += bits[t], nz += bits[t] != 0;
     L->n_sz = 64u * nz;
     L->bit_total = total;
-    int64_t units = (int64_t)((total + kMinUnitBits - 1) / kMinUnitBits);
-    units = std::max<int64_t>(1, std::min<int64_t>(units, std::min<int64_t>(kMaxUnits, T)));
+
+    // decode runs: cut the cost prefix into about equal parts, drop empty runs
+    std::vector<uint64_t> pre((size_t)T + 1, 0);
+    for (int64_t t = 0; t < T; ++t) pre[(size_t)t + 1] = pre[(size_t)t] + block_cost(bits[t]);
+    const uint64_t cost = pre[(size_t)T];
+    int64_t want = (int64_t)((cost + kMinUnitCost - 1) / kMinUnitCost);
+    want = std::max<int64_t>(1, std::min<int64_t>(want, std::min<int64_t>(kMaxUnits, T)));
+    std::vector<uint32_t> bounds;
+    bounds.reserve((size_t)want + 1);
+    bounds.push_back(0u);
+    for (int64_t u = 1; u < want; ++u) {
+        // run u starts at the first block whose cost prefix reaches u*cost/want
+        const uint64_t target = (uint64_t)((unsigned __int128)u * cost / (uint64_t)want);
+        const uint32_t tb = (uint32_t)(std::lower_bound(pre.begin(), pre.begin() + T, target) - pre.begin());
+        if (tb > bounds.back() && tb < (uint32_t)T) bounds.push_back(tb);
+    }
+    bounds.push_back((uint32_t)T);
+    const int64_t units = (int64_t)bounds.size() - 1;
     L->n_units = (int32_t)units;
+    if (sched_words_of(units, T) >= (1ull << 31)) return MPQ_ERR_SHAPE;
+    L->sched_words = (int32_t)sched_words_of(units, T);
+
     if (table) {
         table->assign((size_t)T, mpq_block{0, 0, 0, 0});
-        uint64_t seen[9] = {0}, k = 0, pre = 0;
+        uint64_t seen[9] = {0}, k = 0, bp = 0;
         for (int64_t t = 0; t < T; ++t) {
             const int b = bits[t];
             mpq_block& e = (*table)[(size_t)t];
-            e.bit_prefix = (uint32_t)pre;
+            e.bit_prefix = (uint32_t)bp;
             if (b) {
                 e.code_off = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
                 e.sz_off = (uint32_t)(64u * k);
@@ -75,20 +109,50 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
                 ++seen[b];
                 ++k;
             }
-            pre += (uint64_t)b;
+            bp += (uint64_t)b;
         }
     }
     if (sched) {
-        // unit u starts at the first block whose bit prefix reaches floor(u*S/P)
-        sched->assign((size_t)units + 1, 0u);
-        std::vector<uint64_t> pre((size_t)T + 1, 0);
-        for (int64_t t = 0; t < T; ++t) pre[(size_t)t + 1] = pre[(size_t)t] + bits[t];
-        for (int64_t u = 1; u < units; ++u) {
-            const uint64_t target = (uint64_t)u * total / (uint64_t)units;
-            auto it = std::lower_bound(pre.begin(), pre.begin() + T, target);
-            (*sched)[(size_t)u] = (uint32_t)(it - pre.begin());
+        sched->assign((size_t)L->sched_words, 0u);
+        // runs meeting each block row, and the first partial slot of shared rows
+        std::vector<uint32_t> row_first((size_t)NB, 0u), row_last((size_t)NB, 0u), row_slot((size_t)NB, 0u);
+        for (int64_t u = units - 1; u >= 0; --u)
+            for (uint32_t nb = bounds[(size_t)u] / KB; nb <= (bounds[(size_t)u + 1] - 1) / KB; ++nb)
+                row_first[nb] = (uint32_t)u;
+        for (int64_t u = 0; u < units; ++u)
+            for (uint32_t nb = bounds[(size_t)u] / KB; nb <= (bounds[(size_t)u + 1] - 1) / KB; ++nb)
+                row_last[nb] = (uint32_t)u;
+        uint64_t slots = 0;
+        for (int nb = 0; nb < NB; ++nb) {
+            const uint32_t nc = row_last[nb] - row_first[nb] + 1u;
+            row_slot[nb] = (uint32_t)slots;
+            if (nc > 1) slots += nc;
         }
-        (*sched)[(size_t)units] = (uint32_t)T;
+        uint64_t seen[9] = {0}, k = 0;
+        int64_t t = 0;
+        for (int64_t u = 0; u < units; ++u) {
+            const uint32_t t0 = bounds[(size_t)u], t1 = bounds[(size_t)u + 1];
+            uint32_t* d = sched->data() + (size_t)u * DESC_WORDS;
+            for (; t < t0; ++t) { seen[bits[t]]++; k += bits[t] != 0; }
+            d[DW_T0] = t0;
+            d[DW_T1] = t1;
+            d[DW_SZ] = (uint32_t)(64u * k);
+            for (int i = 0; i < 7; ++i) {
+                const int b = order[i];
+                d[DW_CODE + width_index(b)] = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
+            }
+            const uint32_t ra = t0 / KB, rb = (t1 - 1) / KB;
+            d[DW_A_SLOT] = row_slot[ra];
+            d[DW_A_NC] = row_last[ra] - row_first[ra] + 1u;
+            d[DW_A_IDX] = (uint32_t)u - row_first[ra];
+            d[DW_B_SLOT] = row_slot[rb];
+            d[DW_B_NC] = row_last[rb] - row_first[rb] + 1u;
+            d[DW_B_IDX] = (uint32_t)u - row_first[rb];
+            uint8_t* ib = reinterpret_cast<uint8_t*>(d + DW_BITS);
+            for (uint32_t j = 0; j < (uint32_t)DESC_INLINE_BITS && t0 + j < t1; ++j) ib[j] = bits[t0 + j];
+        }
+        uint8_t* b8 = reinterpret_cast<uint8_t*>(sched->data() + (size_t)units * DESC_WORDS);
+        for (int64_t i = 0; i < T; ++i) b8[i] = bits[i];
     }
     return MPQ_OK;
 }
@@ -125,10 +189,12 @@ LinearWs carve_linear(void* ws, const mpq_layer* layer, int32_t M) {
     w.tok_scale = reinterpret_cast<float*>(base + off);
     off += round256((size_t)M * 4);
     w.xq = reinterpret_cast<__half*>(base + off);
-    // decode: [KB][M][XQD_SLICE]; tensor-core path: [M][K] fp16 (smaller)
-    off += round256((size_t)(layer->K / 128) * M * XQD_SLICE);
+    // decode: [KB][XQD_REC * M]; tensor-core path: [M][K] fp16 (smaller)
+    off += round256((size_t)(layer->K / 128) * M * XQD_REC);
+    // partial sums of shared block rows: at most n_units + NB slots of
+    // 64 rows x (tokens per launch)
     w.partial = reinterpret_cast<float*>(base + off);
-    off += round256((size_t)2 * layer->n_units * 64 * 8 * 4);
+    off += round256((size_t)(layer->n_units + NB) * 64 * std::min(M, kMaxDecodeTokens) * 4);
     w.bytes = off;
     return w;
 }
@@ -153,6 +219,7 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
     return e;
 }
 std::atomic<uint64_t> g_decode_attr{0};
+std::atomic<uint64_t> g_decode_attr8{0};
 std::atomic<uint64_t> g_prefill_attr{0};
 
 // cuTensorMapEncodeTiled from the driver, looked up through the runtime.
@@ -195,6 +262,17 @@ mpq_status mpq_plan(int32_t N, int32_t K, const uint8_t* bits_host, mpq_layout* 
     return make_plan(N, K, bits_host, out, nullptr, nullptr);
 }
 
+mpq_status mpq_plan_schedule(const mpq_layout* L, const uint8_t* bits_host, uint32_t* sched_host) {
+    if (!L || !bits_host || !sched_host) return MPQ_ERR_ARG;
+    mpq_layout chk;
+    std::vector<uint32_t> sched;
+    mpq_status st = make_plan(L->N, L->K, bits_host, &chk, nullptr, &sched);
+    if (st != MPQ_OK) return st;
+    if (chk.n_units != L->n_units || chk.sched_words != L->sched_words) return MPQ_ERR_ARG;
+    std::memcpy(sched_host, sched.data(), sched.size() * 4);
+    return MPQ_OK;
+}
+
 size_t mpq_pack_workspace_size(const mpq_layout*) { return 256; }
 
 mpq_status mpq_pack(const mpq_layout* L, const void* W_dev, const uint8_t* bits_host,
@@ -206,7 +284,8 @@ mpq_status mpq_pack(const mpq_layout* L, const void* W_dev, const uint8_t* bits_
     std::vector<uint32_t> sched;
     mpq_status st = make_plan(L->N, L->K, bits_host, &chk, &table, &sched);
     if (st != MPQ_OK) return st;
-    if (chk.codes_bytes != L->codes_bytes || chk.n_sz != L->n_sz || chk.n_units != L->n_units)
+    if (chk.codes_bytes != L->codes_bytes || chk.n_sz != L->n_sz || chk.n_units != L->n_units ||
+        chk.sched_words != L->sched_words)
         return MPQ_ERR_ARG;
     if (out->N != L->N || out->K != L->K || out->n_units != L->n_units) return MPQ_ERR_ARG;
     if (row_perm_host && !perm_ok(row_perm_host, L->N)) return MPQ_ERR_PERM;
@@ -346,12 +425,13 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         return MPQ_OK;
     }
 
-    e = ensure_smem_attr(k_decode, (int)sizeof(DecSmem), g_decode_attr);
+    e = ensure_smem_attr(k_decode<true>, (int)sizeof(DecSmem), g_decode_attr);
+    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<false>, (int)sizeof(DecSmem), g_decode_attr8);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
     DecodeParams dp{};
     dp.codes = static_cast<const uint8_t*>(layer->codes);
-    dp.table = layer->table;
-    dp.sched = layer->sched;
+    dp.desc = layer->sched;
+    dp.bits8 = reinterpret_cast<const uint8_t*>(layer->sched + (size_t)layer->n_units * DESC_WORDS);
     dp.scales = layer->scales;
     dp.zeros = layer->zeros;
     dp.row_perm = layer->row_perm;
@@ -368,7 +448,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     dp.n_units = layer->n_units;
 
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)layer->n_units);
+    cfg.gridDim = dim3((unsigned)((layer->n_units + DEC_WARPS - 1) / DEC_WARPS));
     cfg.blockDim = dim3(DEC_THREADS);
     cfg.dynamicSmemBytes = sizeof(DecSmem);
     cfg.stream = s;
@@ -382,7 +462,8 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     for (int m0 = 0; m0 < M; m0 += kMaxDecodeTokens) {
         dp.m0 = m0;
         dp.Mg = std::min(kMaxDecodeTokens, M - m0);
-        e = cudaLaunchKernelEx(&cfg, k_decode, dp);
+        e = dp.Mg == 1 ? cudaLaunchKernelEx(&cfg, k_decode<true>, dp)
+                       : cudaLaunchKernelEx(&cfg, k_decode<false>, dp);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
     }
     if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)

@@ -44,9 +44,14 @@
  *   scales, zeros -- fp16 bit patterns, 64 per non-zero block, in ascending t;
  *              row r of block t is at table[t].sz_off + r.
  *   table   -- one mpq_block per block (ascending t).
- *   sched   -- n_units+1 block ids: decode work unit u covers blocks
- *              [sched[u], sched[u+1]) in row-major order, cut so that every
- *              unit holds about the same number of code bytes.
+ *   sched   -- the decode schedule, sched_words 32-bit words: the blocks are
+ *              cut into n_units row-major runs [t0, t1) of about equal
+ *              estimated cost (bytes streamed plus decode work by width),
+ *              one per decode warp.  Run u has a 32-word descriptor at word
+ *              32u: t0, t1, the scale/zero index and the code offset of its
+ *              first block of each width, the partial-sum slots of its
+ *              first and last block rows, and the widths of its first 64
+ *              blocks.  After the descriptors: one byte per block, its width.
  *
  * Conventions:
  *   - The caller owns every buffer.  The library allocates no device memory
@@ -94,8 +99,8 @@ typedef struct {
 /* Sizes of a packed layer; filled by mpq_plan. */
 typedef struct {
     int32_t N, K, NB, KB;    /* NB = N/64, KB = K/128                          */
-    int32_t n_units;         /* decode work units (sched has n_units+1 entries) */
-    int32_t reserved;
+    int32_t n_units;         /* decode work units (runs)                        */
+    int32_t sched_words;     /* 32-bit words of sched                          */
     uint64_t codes_bytes;    /* = 1024 * bit_total                              */
     uint64_t n_sz;           /* = 64 * number of non-zero blocks                */
     uint64_t bit_total;      /* sum of the per-block bits                       */
@@ -111,7 +116,7 @@ typedef struct {
     int32_t reserved;
     const void* codes;           /* uint8  [codes_bytes]                        */
     const mpq_block* table;      /* [NB*KB]                                      */
-    const uint32_t* sched;       /* [n_units + 1]                                */
+    const uint32_t* sched;       /* [sched_words] (mpq_layout)                    */
     const uint16_t* scales;      /* fp16 bits [n_sz]                             */
     const uint16_t* zeros;       /* fp16 bits [n_sz]                             */
     const int32_t* row_perm;     /* int32 [N]; NULL = identity                   */
@@ -125,6 +130,13 @@ typedef struct {
  * Errors: MPQ_ERR_ARG, MPQ_ERR_SHAPE, MPQ_ERR_BITS. */
 mpq_status mpq_plan(int32_t N, int32_t K, const uint8_t* bits_host,
                     mpq_layout* out);
+
+/* Host only.  Writes the decode schedule that mpq_pack stores in `sched`
+ * (sched_words words, format above) for layout L and the same bit map into
+ * host memory, e.g. to inspect the work split.  Errors: ARG (L does not
+ * belong to these bits), SHAPE, BITS. */
+mpq_status mpq_plan_schedule(const mpq_layout* L, const uint8_t* bits_host,
+                             uint32_t* sched_host);
 
 /* Workspace bytes that mpq_pack needs (the error word). */
 size_t mpq_pack_workspace_size(const mpq_layout* L);
@@ -158,8 +170,10 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
  *   y_dev   fp32, M x N row-major, original output order (device).
  *   ws      device workspace of >= mpq_linear_workspace_size(layer, M) bytes,
  *           256-byte aligned; its contents need no initialization.
- * Uses a memory-bound decode kernel for M <= 32 and a tensor-core kernel for
- * larger M.  Non-finite x gives non-finite y (no error).
+ * Uses a memory-bound decode kernel for M <= 16 and a tensor-core kernel for
+ * larger M.  Non-finite x gives non-finite y (no error).  Activations are
+ * moved into fp16 by exact powers of two; for M <= 16 that needs
+ * |x| < 2^118 (larger magnitudes overflow to inf).
  * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT. */
 mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M,
                       float* y_dev, void* ws, size_t ws_bytes, void* stream);
