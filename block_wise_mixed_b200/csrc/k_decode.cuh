@@ -76,6 +76,7 @@ struct DecodeParams {
 
 constexpr int DEC_WARPS = 4;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
+constexpr int DEC_CTAS_PER_SM = 4;   // 16 resident warps per SM
 constexpr int DEC_RING = 12288;      // bytes of ring per warp (>= largest stage)
 constexpr int DEC_SLOTS = 8;         // stages in flight per warp
 constexpr int DEC_MAX_TOKENS = 8;
@@ -89,10 +90,10 @@ struct DecSmem {
     DecWarp w[DEC_WARPS];
 };
 
-// 4 CTAs per SM: 4 x (smem + 1 KB reserved) must fit the SM's 228 KB
-static_assert(4 * (sizeof(DecSmem) + 1024) <= 228 * 1024, "decode smem too large for 4 CTAs/SM");
+// DEC_CTAS_PER_SM x (smem + 1 KB reserved) must fit the SM's 228 KB
+static_assert(DEC_CTAS_PER_SM * (sizeof(DecSmem) + 1024) <= 228 * 1024, "decode smem too large");
 // largest stage: an 8-bit payload
-static_assert(DEC_RING >= 8 * 1024 + 256 + DEC_MAX_TOKENS * (XQD_VAR + XQD_AUX), "ring too small");
+static_assert(DEC_RING >= 8 * 1024 + 256 + DEC_MAX_TOKENS * XQD_VAR, "ring too small");
 
 __host__ __device__ constexpr int lo_width(int b) { return (b == 3) ? 2 : (b == 5 || b == 6) ? 4 : b; }
 __host__ __device__ constexpr int hi_width(int b) { return (b == 3 || b == 5) ? 1 : (b == 6) ? 2 : 0; }
@@ -230,30 +231,54 @@ __device__ __forceinline__ void row_pairs(const uint8_t* stage, int r, int t, ui
     }
 }
 
-// cg[rt][*] = 2^-24 * sum over the block's 128 columns of (q - z) * x'
-// (C-fragment order: rows 16rt+g, 16rt+g+8 x tokens 2t, 2t+1).
-template <int B>
-__device__ __forceinline__ void block_mma(const uint8_t* stage, const uint32_t (&b)[16],
-                                          float (&cg)[4][4], int g, int t) {
-    const uint16_t* zr16 = reinterpret_cast<const uint16_t*>(stage + 1024 * B) + 64;
+// One 16-row tile rt of a block of width B, added into acc:
+//   c = 2^-24 * sum over the block's 128 columns of (q - z) * x'
+//   acc[rt][*] += s_row * F_tok * c        (C-fragment order: rows 16rt+g,
+//   16rt+g+8 x tokens 2t, 2t+1).
+// The caller loops over rt at run time, so each width's code is one tile's
+// worth (small enough to stay in the instruction cache); the tile's eight
+// k-steps alternate between two accumulators to halve the mma chain.
+template <int B, bool ONE_TOKEN>
+__device__ __forceinline__ void tile_accumulate(const uint8_t* stage, const uint32_t (&b)[16], int rt,
+                                                int g, int t, float Fa, float Fb, float (&acc)[4][4]) {
+    const uint16_t* sc16 = reinterpret_cast<const uint16_t*>(stage + 1024 * B);
+    const int r0 = 16 * rt + g, r1 = r0 + 8;
+    // -z * 2^-24 in both halves (z is an fp16 integer; 0x8001 = -2^-24)
+    const uint32_t zc0 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)sc16[64 + r0], 0u, 0x1010)),
+                                         bits_h2(0x80018001u)));
+    const uint32_t zc1 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)sc16[64 + r1], 0u, 0x1010)),
+                                         bits_h2(0x80018001u)));
+    uint32_t a0[16], a1[16];
+    row_pairs<B>(stage, r0, t, zc0, a0);
+    row_pairs<B>(stage, r1, t, zc1, a1);
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-        const int r0 = 16 * rt + g, r1 = r0 + 8;
-        // zc = -z * 2^-24 in both halves (z is an fp16 integer; 0x8001 = -2^-24)
-        const uint32_t zc0 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)zr16[r0], 0u, 0x1010)),
-                                             bits_h2(0x80018001u)));
-        const uint32_t zc1 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)zr16[r1], 0u, 0x1010)),
-                                             bits_h2(0x80018001u)));
-        uint32_t a0[16], a1[16];
-        row_pairs<B>(stage, r0, t, zc0, a0);
-        row_pairs<B>(stage, r1, t, zc1, a1);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            mma_16816(c, a0[2 * ks], a1[2 * ks], a0[2 * ks + 1], a1[2 * ks + 1], b[2 * ks], b[2 * ks + 1]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) cg[rt][k] = c[k];
+    for (int ks = 0; ks < 8; ks += 2) {
+        mma_16816(c, a0[2 * ks], a1[2 * ks], a0[2 * ks + 1], a1[2 * ks + 1], b[2 * ks], b[2 * ks + 1]);
+        mma_16816(d, a0[2 * ks + 2], a1[2 * ks + 2], a0[2 * ks + 3], a1[2 * ks + 3], b[2 * ks + 2],
+                  b[2 * ks + 3]);
     }
+    const float s0 = __half2float(__ushort_as_half(sc16[r0]));
+    const float s1 = __half2float(__ushort_as_half(sc16[r1]));
+    const float v0 = s0 * (Fa * (c[0] + d[0]));
+    const float v2 = s1 * (Fa * (c[2] + d[2]));
+    const float v1 = ONE_TOKEN ? 0.f : s0 * (Fb * (c[1] + d[1]));
+    const float v3 = ONE_TOKEN ? 0.f : s1 * (Fb * (c[3] + d[3]));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {   // acc[rt] without run-time register indexing
+        if (k == rt) {
+            acc[k][0] += v0;
+            acc[k][2] += v2;
+            if (!ONE_TOKEN) { acc[k][1] += v1; acc[k][3] += v3; }
+        }
+    }
+}
+
+template <int B, bool ONE_TOKEN>
+__device__ __forceinline__ void block_accumulate(const uint8_t* stage, const uint32_t (&b)[16], int g,
+                                                 int t, float Fa, float Fb, float (&acc)[4][4]) {
+#pragma unroll 1
+    for (int rt = 0; rt < 4; ++rt) tile_accumulate<B, ONE_TOKEN>(stage, b, rt, g, t, Fa, Fb, acc);
 }
 
 __device__ __forceinline__ void load_bfrag(const uint8_t* src, uint32_t (&b)[16]) {
@@ -266,10 +291,10 @@ __device__ __forceinline__ void load_bfrag(const uint8_t* src, uint32_t (&b)[16]
 }
 
 // Stage layout in the ring (all parts 16-byte multiples):
-//   payload 1024*b | scales 128 | zeros 128 | x' variant of the low piece
-//   256*Mg | F 16*Mg
+//   payload 1024*b | scales 128 | zeros 128 | x' variant of the low piece,
+//   272 bytes per token (fragments, then F)
 __device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
-    return 1024u * b + 256u + (XQD_VAR + XQD_AUX) * Mg;
+    return 1024u * b + 256u + XQD_VAR * Mg;
 }
 
 // ---------------------------------------------------------------------------
@@ -277,7 +302,7 @@ __device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
 // carries data, so the per-block epilogue handles half the elements).
 // ---------------------------------------------------------------------------
 template <bool ONE_TOKEN>
-__global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
+__global__ void __launch_bounds__(DEC_THREADS, DEC_CTAS_PER_SM) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -287,6 +312,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
     const uint32_t KB = (uint32_t)p.KB;
     const uint32_t lt_mask = (1u << lane) - 1u;
 
+    // the next kernel in the stream may launch now: it waits (griddepcontrol)
+    // for this grid before it touches memory this kernel uses
+    pdl_launch_dependents();
     if (lane == 0) {
         for (int s = 0; s < DEC_SLOTS; ++s) mbar_init(&W.full[s], 1);
         fence_mbar_init();
@@ -303,14 +331,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
     // lanes DW_CODE..DW_CODE+6 keep the running code offset of their width
     uint32_t code_run = dw;
 
+
     const uint32_t Mg = (uint32_t)p.Mg;
-    const size_t rec_bytes = (size_t)p.M_total * XQD_REC;
-    const uint8_t* xq_tok = p.xq + (size_t)p.m0 * XQD_VAR;     // + kb*rec + v*M*256
-    const uint8_t* xq_aux = p.xq + (size_t)4 * p.M_total * XQD_VAR + (size_t)p.m0 * XQD_AUX;
+    // xq offsets fit 32 bits: KB * M * XQD_REC < 2^32 (the host checks it)
+    const uint32_t rec_bytes = (uint32_t)p.M_total * XQD_REC;
+    const uint32_t var_bytes = (uint32_t)p.M_total * XQD_VAR;
+    const uint32_t x_tok_off = (uint32_t)p.m0 * XQD_VAR;
+    const uint32_t x_bytes = XQD_VAR * Mg;
 
     // ---- chunk state: lane l describes block t0 + 32*chunk + l ----
     uint32_t chunk = 0;
-    uint32_t c_bits = 0, c_code = 0, c_sz = 0;
+    uint32_t c_bits = 0, c_code = 0, c_sz = 0, c_x = 0;
     uint32_t pending = 0;            // non-zero blocks of the chunk not yet issued
     bool scan_done = false;
     uint32_t bits_pref = 0;          // prefetched widths of the next chunk (beyond the inline 64)
@@ -328,6 +359,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
         const uint32_t jn = j + 32u;
         if (jn >= (uint32_t)DESC_INLINE_BITS && t0 + jn < t1) bits_pref = __ldg(p.bits8 + t0 + jn);
         c_bits = b;
+        // this block's activation variant for the launch's tokens, as a byte
+        // offset into xq (one division per chunk instead of one per stage)
+        c_x = ((t0 + j) % KB) * rec_bytes + (uint32_t)variant_of(lo_width(b == 0 ? 1 : (int)b)) * var_bytes +
+              x_tok_off;
         // rank among the chunk's blocks of the same width -> code offset
         const uint32_t same = __match_any_sync(0xffffffffu, b);
         const uint32_t rank = __popc(same & lt_mask);
@@ -357,17 +392,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
     uint32_t q_head = 0, q_tail = 0;     // consumed / issued stages
     uint32_t r_head = 0, r_tail = 0;     // ring bytes issued / freed (monotone)
     uint32_t r_pos = 0;                  // physical ring offset of r_head
-    uint32_t qe_t = 0, qe_bits = 0, qe_off = 0, qe_end = 0;
+    uint32_t qe_t = 0, qe_bits = 0, qe_off = 0, qe_end = 0, qe_x = 0;
     bool xq_ready = false;               // x' is written by the prologue kernel
-
-    auto issue_x = [&](uint32_t tt, uint32_t b, uint32_t off, uint32_t slot) {
-        const uint32_t kb = tt % KB;
-        uint8_t* dst = W.ring + off + 1024u * b + 256u;
-        const uint8_t* rec = xq_tok + (size_t)kb * rec_bytes;
-        const uint32_t vb = XQD_VAR * Mg;
-        bulk_g2s(dst, rec + (size_t)variant_of(lo_width((int)b)) * p.M_total * XQD_VAR, vb, &W.full[slot]);
-        bulk_g2s(dst + vb, xq_aux + (size_t)kb * rec_bytes, XQD_AUX * Mg, &W.full[slot]);
-    };
     auto issue_more = [&]() {
         while (q_tail - q_head < (uint32_t)DEC_SLOTS && !scan_done) {
             if (aborted) { scan_done = true; break; }
@@ -383,7 +409,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
             const uint32_t b = __shfl_sync(0xffffffffu, c_bits, l);
             const uint32_t coff = __shfl_sync(0xffffffffu, c_code, l);
             const uint32_t szo = __shfl_sync(0xffffffffu, c_sz, l);
-            const uint32_t size = stage_bytes(b, Mg);
+            const uint32_t xo = __shfl_sync(0xffffffffu, c_x, l);
+            const uint32_t size = 1024u * b + 256u + x_bytes;   // stage_bytes(b, Mg)
             // a stage never wraps: when the ring's tail end is too short, skip to 0
             const bool skip = r_pos + size > (uint32_t)DEC_RING;
             const uint32_t start = skip ? r_head + ((uint32_t)DEC_RING - r_pos) : r_head;
@@ -399,9 +426,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
                 bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
                 bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
                 bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
-                if (xq_ready) issue_x(tt, b, off, slot);
+                if (xq_ready) bulk_g2s(dst + 1024u * b + 256u, p.xq + xo, x_bytes, bar);
             }
-            if (lane == (int)slot) { qe_t = tt; qe_bits = b; qe_off = off; qe_end = start + size; }
+            if (lane == (int)slot) { qe_t = tt; qe_bits = b; qe_off = off; qe_end = start + size; qe_x = xo; }
             r_head = start + size;
             r_pos = off + size;
             ++q_tail;
@@ -416,10 +443,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
     xq_ready = true;
     for (uint32_t k = q_head; k < q_tail; ++k) {
         const uint32_t slot = k % DEC_SLOTS;
-        const uint32_t kt = __shfl_sync(0xffffffffu, qe_t, slot);
         const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
         const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
-        if (lane == 0) issue_x(kt, kbits, ko, slot);
+        const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
+        if (lane == 0) bulk_g2s(W.ring + ko + 1024u * kbits + 256u, p.xq + kx, x_bytes, &W.full[slot]);
     }
 
     const uint32_t nb_first = t0 / KB, nb_last = (t1 - 1) / KB;
@@ -457,35 +484,21 @@ __global__ void __launch_bounds__(DEC_THREADS, 4) k_decode(DecodeParams p) {
             if (!aborted) {
                 const uint8_t* stage = W.ring + foff;
                 const uint8_t* xs = stage + 1024u * fb + 256u;
-                const uint8_t* aux = xs + XQD_VAR * Mg;
                 // this lane's B fragments: token g, quad lane t; zeros beyond Mg
                 uint32_t bf[16];
                 load_bfrag((uint32_t)g < Mg ? xs + g * XQD_VAR + t * 64
                                             : reinterpret_cast<const uint8_t*>(W.zero16), bf);
-                float cg[4][4];
-                switch (fb) {
-                    case 1: block_mma<1>(stage, bf, cg, g, t); break;
-                    case 2: block_mma<2>(stage, bf, cg, g, t); break;
-                    case 3: block_mma<3>(stage, bf, cg, g, t); break;
-                    case 4: block_mma<4>(stage, bf, cg, g, t); break;
-                    case 5: block_mma<5>(stage, bf, cg, g, t); break;
-                    case 6: block_mma<6>(stage, bf, cg, g, t); break;
-                    default: block_mma<8>(stage, bf, cg, g, t); break;
-                }
-                // epilogue: acc += s * F * cg per row and token
-                const uint16_t* sc16 = reinterpret_cast<const uint16_t*>(stage + 1024u * fb);
-                const float Fa = (2u * t < Mg) ? *reinterpret_cast<const float*>(aux + (2 * t) * XQD_AUX) : 0.f;
+                const float Fa = (2u * t < Mg) ? *reinterpret_cast<const float*>(xs + (2 * t) * XQD_VAR + 256) : 0.f;
                 const float Fb = (!ONE_TOKEN && 2u * t + 1u < Mg)
-                                     ? *reinterpret_cast<const float*>(aux + (2 * t + 1) * XQD_AUX) : 0.f;
-#pragma unroll
-                for (int rt = 0; rt < 4; ++rt) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float sr = __half2float(__ushort_as_half(sc16[16 * rt + 8 * h + g]));
-                        // F * cg is the block's sum at the activations' own scale
-                        acc[rt][2 * h] = fmaf(sr, Fa * cg[rt][2 * h], acc[rt][2 * h]);
-                        if (!ONE_TOKEN) acc[rt][2 * h + 1] = fmaf(sr, Fb * cg[rt][2 * h + 1], acc[rt][2 * h + 1]);
-                    }
+                                     ? *reinterpret_cast<const float*>(xs + (2 * t + 1) * XQD_VAR + 256) : 0.f;
+                switch (fb) {
+                    case 1: block_accumulate<1, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    case 2: block_accumulate<2, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    case 3: block_accumulate<3, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    case 4: block_accumulate<4, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    case 5: block_accumulate<5, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    case 6: block_accumulate<6, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    default: block_accumulate<8, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
                 }
             }
             __syncwarp();

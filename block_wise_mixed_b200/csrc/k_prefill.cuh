@@ -211,6 +211,9 @@ __device__ __forceinline__ void dequant_row_half(const uint8_t* payload, const _
 __global__ void __launch_bounds__(PF_THREADS, 1)
 k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // the next kernel may launch once every CTA of this grid has started; it
+    // waits (griddepcontrol.wait) for this grid before touching its memory
+    pdl_launch_dependents();
     // the operand tiles need 1024-byte alignment (128B swizzle atoms)
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(base);

@@ -43,8 +43,10 @@ constexpr int XPREP_THREADS = 256;
 
 template <int LAYOUT>
 __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
-    // let the GEMM kernel that follows start its prologue early
+    // let the GEMM kernel that follows start its prologue early, then wait
+    // for the kernel before (x and the workspace may still be in use there)
     pdl_launch_dependents();
+    pdl_wait();
     __shared__ float red[XPREP_THREADS / 32];
     const int m = blockIdx.x, tid = threadIdx.x, K = p.K;
     if (m == 0) {
@@ -134,16 +136,15 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
 // c_r = 2^-24 * sum_j (q_j - z_r) x'_j, and the block adds s_r * F * c_r to
 // output row r, with F = 2^(24 - e).
 //
-// Record of block column kb (XQD_REC * M bytes, 16-byte aligned):
-//   [v = 0..3 (p = 1, 2, 4, 8)][m][t = 0..3][pi = 0..15] half2   (4*256*M B)
-//   [m] float4 (F, 0, 0, 0)                                       (16*M B)
-// so one variant of a token group is one contiguous run of 256*Mg bytes.
+// Record of block column kb (XQD_REC * M bytes, 16-byte aligned): for each
+// variant v = 0..3 (p = 1, 2, 4, 8) and token m, XQD_VAR = 272 bytes:
+//   [t = 0..3][pi = 0..15] half2 (256 B), then F as float4 (F, 0, 0, 0)
+// so one variant of a token group is one contiguous run of 272*Mg bytes.
 // Block 0 also clears the workspace error word and the decode kernel's
 // per-block-row counters.
 // ---------------------------------------------------------------------------
-constexpr int XQD_VAR = 256;                 // one variant of one token
-constexpr int XQD_AUX = 16;                  // F of one token (padded)
-constexpr int XQD_REC = 4 * XQD_VAR + XQD_AUX;
+constexpr int XQD_VAR = 272;                 // one variant of one token: fragments + F
+constexpr int XQD_REC = 4 * XQD_VAR;
 
 __device__ __forceinline__ void xqd_pair_cols(int v, int pi, int& ca, int& cb) {
     if (v == 0) {
@@ -161,6 +162,7 @@ constexpr int XPREP_DEC_WARPS = XPREP_THREADS / 32;
 
 __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
     pdl_launch_dependents();
+    pdl_wait();   // the kernel before may still read the workspace or write x
     __shared__ float xs[XPREP_DEC_WARPS][64];   // 128 fp16 per warp
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int KB = p.K / 128;
@@ -221,8 +223,8 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
                                           tq * 64 + pi0 * 4);
     dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
     dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-    if (lane == 0)
-        *reinterpret_cast<float4*>(rec + (size_t)4 * p.M * XQD_VAR + (size_t)m * XQD_AUX) =
+    if ((lane & 7) == 0)   // one lane per variant writes F after the fragments
+        *reinterpret_cast<float4*>(rec + (size_t)vv * p.M * XQD_VAR + (size_t)m * XQD_VAR + 256) =
             make_float4(ldexpf(1.f, 24 - e), 0.f, 0.f, 0.f);
 }
 

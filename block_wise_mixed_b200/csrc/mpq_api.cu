@@ -22,7 +22,7 @@ using namespace mpq;
 
 namespace {
 
-constexpr int kMaxUnits = 148 * 16;    // one run per resident decode warp (16 per SM)
+constexpr int kMaxUnits = 148 * DEC_CTAS_PER_SM * DEC_WARPS;   // one run per resident decode warp
 constexpr uint64_t kMinUnitCost = 4096; // cost units (bytes) per run, at least
 constexpr int kMaxDecodeTokens = DEC_MAX_TOKENS;   // tokens per decode launch
 constexpr int kDecodeMaxM = 16;         // larger batches take the tensor-core kernel
@@ -363,6 +363,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     const int NB = layer->N / 64, KB = layer->K / 128;
 
     const bool use_tc = M > kDecodeMaxM;
+    if (!use_tc && (uint64_t)KB * (uint64_t)M * XQD_REC >= (1ull << 32)) return MPQ_ERR_SHAPE;
     XprepParams xp{};
     xp.x = static_cast<const uint16_t*>(x_dev);
     xp.col_perm = layer->col_perm;
@@ -373,19 +374,29 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     xp.err = w.err;
     xp.M = M;
     xp.K = layer->K;
-    if (use_tc) {
-        xp.counters = nullptr;
-        k_xprep<XP_PREFILL><<<M, XPREP_THREADS, 0, s>>>(xp);
-    } else {
-        const int items = KB * M, per = XPREP_THREADS / 32;
-        k_xprep_decode<<<(items + per - 1) / per, XPREP_THREADS, 0, s>>>(xp);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return MPQ_ERR_CUDA;
-
+    // Every launch may overlap the end of the kernel before it (programmatic
+    // dependent launch): each kernel waits (griddepcontrol.wait) for its
+    // predecessor before it touches memory the predecessor uses.
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t xc{};
+    xc.blockDim = dim3(XPREP_THREADS);
+    xc.stream = s;
+    xc.attrs = pdl;
+    xc.numAttrs = 1;
+    cudaError_t e;
+    if (use_tc) {
+        xp.counters = nullptr;
+        xc.gridDim = dim3((unsigned)M);
+        e = cudaLaunchKernelEx(&xc, k_xprep<XP_PREFILL>, xp);
+    } else {
+        const int items = KB * M, per = XPREP_THREADS / 32;
+        xc.gridDim = dim3((unsigned)((items + per - 1) / per));
+        e = cudaLaunchKernelEx(&xc, k_xprep_decode, xp);
+    }
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+
     if (use_tc) {
         const size_t smem = prefill_smem_bytes(KB);
         if (smem > 227 * 1024) return MPQ_ERR_SHAPE;
