@@ -77,12 +77,14 @@ struct DecodeParams {
 constexpr int DEC_WARPS = 4;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
 constexpr int DEC_CTAS_PER_SM = 4;   // 16 resident warps per SM
+constexpr int DEC_MAX_REGS = 112;
 constexpr int DEC_RING = 12288;      // bytes of ring per warp (>= largest stage)
 constexpr int DEC_SLOTS = 8;         // stages in flight per warp
 constexpr int DEC_MAX_TOKENS = 8;
 
 struct DecWarp {
     uint8_t ring[DEC_RING];
+    int32_t rows[64];         // output index of each row of the current block row
     uint64_t full[DEC_SLOTS];
     uint4 zero16[4];          // zero B fragments for lanes beyond the token count
 };
@@ -297,12 +299,62 @@ __device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
     return 1024u * b + 256u + XQD_VAR * Mg;
 }
 
+// Last arriver of a shared block row: y[m][rows[r]] = sum over the row's nc
+// runs (in run order) of their partial sums.  The slots are contiguous
+// ([nc][Mg tokens][64 rows] floats at `slots`); lanes read float4 vectors of
+// them, eight slots per batch with every load of a batch in flight.  With one
+// token a slot is 16 vectors, so two lane groups take the even and odd slots
+// and are combined in that order (the sum stays deterministic).  Kept out of
+// line: it runs once per shared row, and its registers must not weigh on the
+// block loop.
+__device__ __noinline__ void finish_shared_row(const float* __restrict__ slots, uint32_t Mg, uint32_t nc,
+                                               float* __restrict__ y, int N, const int32_t* rows, int lane) {
+    const float4* pv = reinterpret_cast<const float4*>(slots);
+    const uint32_t V = Mg * 16u;
+    const uint32_t groups = (V == 16u) ? 2u : 1u;
+    const uint32_t grp = (V == 16u) ? (uint32_t)lane >> 4 : 0u;
+    for (uint32_t v = (V == 16u) ? ((uint32_t)lane & 15u) : (uint32_t)lane; v < V; v += 32u) {
+        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (uint32_t c0 = grp; c0 < nc; c0 += 8u * groups) {
+            float4 q[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t c = c0 + (uint32_t)k * groups;
+                q[k] = c < nc ? __ldcg(pv + (size_t)c * V + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                tot.x += q[k].x; tot.y += q[k].y; tot.z += q[k].z; tot.w += q[k].w;
+            }
+        }
+        if (groups == 2u) {   // even slots' sum + odd slots' sum
+            const int lo = (int)(v & 15u);
+            float4 all;
+            all.x = __shfl_sync(0xffffffffu, tot.x, lo) + __shfl_sync(0xffffffffu, tot.x, lo + 16);
+            all.y = __shfl_sync(0xffffffffu, tot.y, lo) + __shfl_sync(0xffffffffu, tot.y, lo + 16);
+            all.z = __shfl_sync(0xffffffffu, tot.z, lo) + __shfl_sync(0xffffffffu, tot.z, lo + 16);
+            all.w = __shfl_sync(0xffffffffu, tot.w, lo) + __shfl_sync(0xffffffffu, tot.w, lo + 16);
+            tot = all;
+        }
+        if (grp == 0u) {   // vector v: token v / 16, rows 4 (v % 16) .. +3
+            const uint32_t r = 4u * (v & 15u);
+            float* yr = y + (size_t)(v >> 4) * N;
+            yr[rows[r]] = tot.x;
+            yr[rows[r + 1]] = tot.y;
+            yr[rows[r + 2]] = tot.z;
+            yr[rows[r + 3]] = tot.w;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The kernel.  ONE_TOKEN: the launch has Mg == 1 (only C-fragment column 0
 // carries data, so the per-block epilogue handles half the elements).
 // ---------------------------------------------------------------------------
 template <bool ONE_TOKEN>
-__global__ void __launch_bounds__(DEC_THREADS, DEC_CTAS_PER_SM) k_decode(DecodeParams p) {
+// At most 112 registers: four CTAs then leave room in the register file for
+// the next launch's activation-prologue CTAs to become resident early.
+__global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -551,43 +603,13 @@ __global__ void __launch_bounds__(DEC_THREADS, DEC_CTAS_PER_SM) k_decode(DecodeP
         last = __shfl_sync(0xffffffffu, last, 0);
         __syncwarp();
         if (!last) continue;
-        float tot[4][4];
+        if (t == 0) {   // the row's output indices, for the lanes that write y below
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tot[a][c] = 0.f;
-#pragma unroll 4
-        for (uint32_t c = 0; c < nc; ++c) {
-            // the slots of the row's runs, in run order (deterministic sum)
-            const float* pc = p.partial + (size_t)(slot_base + c) * Mg * 64;
-            float v[4][4];
-#pragma unroll
-            for (int rt = 0; rt < 4; ++rt)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = 16 * rt + 8 * h + g;
-                    v[rt][2 * h] = wa ? __ldcg(pc + tok_a * 64 + r) : 0.f;
-                    v[rt][2 * h + 1] = wb ? __ldcg(pc + tok_b * 64 + r) : 0.f;
-                }
-            if (c == idx) {
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) v[a][cc] = acc[a][cc];
-            }
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tot[a][cc] += v[a][cc];
+            for (int q = 0; q < 8; ++q) W.rows[8 * q + g] = rp[q];
         }
-#pragma unroll
-        for (int rt = 0; rt < 4; ++rt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int n = rp[2 * rt + h];
-                if (wa) p.y[(size_t)(p.m0 + tok_a) * p.N + n] = tot[rt][2 * h];
-                if (wb) p.y[(size_t)(p.m0 + tok_b) * p.N + n] = tot[rt][2 * h + 1];
-            }
+        __syncwarp();
+        finish_shared_row(p.partial + (size_t)slot_base * Mg * 64, Mg, nc, p.y + (size_t)p.m0 * p.N,
+                          p.N, W.rows, lane);
         if (lane == 0) p.counters[nb] = 0u;   // ready for the next launch
     }
 }
