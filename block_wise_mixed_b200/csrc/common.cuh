@@ -77,13 +77,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Waits for the phase with the given parity to complete, for at most about
 // `limit_ns` nanoseconds.  Returns false (and leaves the phase pending) when
-// the limit ran out; the caller records MPQ_ERR_TIMEOUT and winds down.
+// the limit ran out; the caller records MPQ_ERR_TIMEOUT and winds down.  The
+// poll loop is kept tight (the clock is read every 64 polls): waiting warps
+// share the issue slots with the warps that do the work.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }

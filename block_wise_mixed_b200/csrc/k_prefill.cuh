@@ -7,14 +7,17 @@
 // "Key results"); TileQuant's abstract describes the same split -- compact
 // per-tile buffers expanded next to the 16-bit tensor-core computation.
 //
-// Roles (10 warps):
-//   warp 0     producer: 1-D bulk copies of the two blocks' payloads and
-//              scales/zeros per 128-wide k block into a ring, and the x' tile
-//              (TMA tensor copy, 128B swizzle) into the operand stage.
+// Roles (19 warps):
+//   warp 0     producer of the codes: 1-D bulk copies of the two blocks'
+//              payloads and scales/zeros per 128-wide k block, as far ahead as
+//              the code stages allow.
+//   warp 18    producer of the activations: the x' tile of each k block (TMA
+//              tensor copy, 128B swizzle) into its own stages.
 //   warp 1     allocates TMEM and issues tcgen05.mma (one elected thread).
-//   warps 2-9  dequantize: each thread expands half of one weight row's
+//   warps 2-17 dequantize: each thread expands a quarter of one weight row's
 //              128 codes into fp16 w_hat = (q - z) * s, written straight
-//              into the K-major 128B-swizzled shared-memory A operand; after
+//              into the K-major 128B-swizzled shared-memory A operand (four
+//              warps per TMEM lane quadrant keep the schedulers busy); after
 //              the last k block they read the fp32 accumulator out of TMEM
 //              and write y.
 // A k block whose two blocks are both 0-bit is skipped by every role (no
@@ -37,24 +40,27 @@
 
 namespace mpq {
 
-constexpr int PF_WARPS = 10;
+constexpr int PF_DQ_WARPS = 16;                  // warps 2 .. 17
+constexpr int PF_WARPS = PF_DQ_WARPS + 3;
 constexpr int PF_THREADS = PF_WARPS * 32;
-constexpr int PF_DQ_WARPS = 8;
 constexpr int PF_BM = 128;       // weight rows per tile (2 block rows)
 constexpr int PF_BN = 128;       // tokens per tile
-constexpr int PF_AB_STAGES = 2;
-constexpr int PF_C_STAGES = 3;
+constexpr int PF_A_STAGES = 2;   // dequantized weight tiles
+constexpr int PF_B_STAGES = 2;   // activation tiles (from L2)
+constexpr int PF_C_STAGES = 5;   // packed codes (from HBM: the longer latency)
 constexpr int PF_A_BYTES = PF_BM * 256;           // 128 rows x 128 fp16
 constexpr int PF_B_BYTES = PF_BN * 256;           // 128 tokens x 128 fp16
 constexpr int PF_C_BYTES = 2 * 8192 + 4 * 128;    // two payloads + 2 x (scales, zeros)
 constexpr uint32_t PF_TMEM_COLS = 128;
 
 struct PrefillSmem {
-    uint8_t a[PF_AB_STAGES][PF_A_BYTES];   // 1024-aligned (offset 0)
-    uint8_t b[PF_AB_STAGES][PF_B_BYTES];
+    uint8_t a[PF_A_STAGES][PF_A_BYTES];    // 1024-aligned (offset 0)
+    uint8_t b[PF_B_STAGES][PF_B_BYTES];
     uint8_t c[PF_C_STAGES][PF_C_BYTES];
-    uint64_t full_ab[PF_AB_STAGES];
-    uint64_t empty_ab[PF_AB_STAGES];
+    uint64_t full_a[PF_A_STAGES];
+    uint64_t empty_a[PF_A_STAGES];
+    uint64_t full_b[PF_B_STAGES];
+    uint64_t empty_b[PF_B_STAGES];
     uint64_t full_c[PF_C_STAGES];
     uint64_t empty_c[PF_C_STAGES];
     uint64_t d_full;
@@ -71,6 +77,7 @@ struct PrefillParams {
     const int32_t* row_perm;
     const float* tok_scale;   // [M]
     float* y;                 // [M][N]
+    int permuted_out;         // 1: write y in W' row order (k_unpermute_rows fixes it)
     uint32_t* err;
     int N, K, NB, KB, M;
     int tiles_n;              // ceil(NB / 2)
@@ -145,10 +152,31 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int kc) {
                       (((kc & 7) ^ (r & 7)) << 4));
 }
 
-// Dequantizes groups [g0, g0+8) (8 codes each) of row rr of one block of
-// width B into the A tile row r: w_hat = (q - z) * s in fp16.
+// Dequantizes groups [g0, g0+4) (8 codes each) of row rr of one block of
+// width B into the A tile row r: w_hat = (q - z) * s in fp16.  A warp covers
+// 8 whole rows (lane = row * 4 + quarter), so the lanes' code bytes are one
+// contiguous run of shared memory (one conflict-free vector load each), and
+// their 16-byte A chunks fall four to a bank group.
+template <int P>
+__device__ __forceinline__ void load_part(const uint8_t* p, uint32_t (&w)[P]) {
+    if (P == 1) {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else if (P == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = v.x; w[1] = v.y;
+    } else if (P == 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+        const uint4 v0 = reinterpret_cast<const uint4*>(p)[0];
+        const uint4 v1 = reinterpret_cast<const uint4*>(p)[1];
+        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+        w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    }
+}
+
 template <int B>
-__device__ __forceinline__ void dequant_row_half(const uint8_t* payload, const __half* scz, int rr,
+__device__ __forceinline__ void dequant_row_part(const uint8_t* payload, const __half* scz, int rr,
                                                  int g0, uint8_t* a_tile, int r) {
     constexpr int P0 = (B == 3) ? 2 : (B == 5 || B == 6) ? 4 : B;
     constexpr int P1 = (B == 3 || B == 5) ? 1 : (B == 6) ? 2 : 0;
@@ -157,26 +185,17 @@ __device__ __forceinline__ void dequant_row_half(const uint8_t* payload, const _
     const __half2 s2 = __half2half2(sh);
     uint32_t k[4];
     zero_consts<P0>(z2, k);
-    // this half-row's bytes of each piece: groups g0..g0+7 = codes 8*g0 .. 8*g0+63
-    const uint8_t* lo = payload + rr * 16 * P0 + (g0 * 8 * P0) / 8;
-    uint32_t d[2 * P0];   // 64 codes of P0 bits = 8*P0 bytes = 2*P0 words
-#pragma unroll
-    for (int q = 0; q < 2 * P0; q += (P0 >= 2 ? 2 : 1)) {
-        if (P0 >= 2) {
-            uint2 v = *reinterpret_cast<const uint2*>(lo + 4 * q);
-            d[q] = v.x; d[q + 1] = v.y;
-        } else {
-            d[q] = *reinterpret_cast<const uint32_t*>(lo + 4 * q);
-        }
-    }
-    uint32_t e[P1 > 0 ? 2 * P1 : 1];
-    if (P1 > 0) {
-        const uint8_t* hi = payload + 64 * 16 * P0 + rr * 16 * P1 + (g0 * 8 * P1) / 8;
-#pragma unroll
-        for (int q = 0; q < 2 * P1; ++q) e[q] = *reinterpret_cast<const uint32_t*>(hi + 4 * q);
+    // the part's 32 codes: 4*P0 bytes of the low piece, 4*P1 of the high one
+    uint32_t d[P0];
+    load_part<P0>(payload + rr * 16 * P0 + g0 * P0, d);
+    uint32_t e[P1 > 0 ? P1 : 1];
+    if (P1 == 1) e[0] = *reinterpret_cast<const uint32_t*>(payload + 64 * 16 * P0 + rr * 16 + g0);
+    if (P1 == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(payload + 64 * 16 * P0 + rr * 32 + 2 * g0);
+        e[0] = v.x; e[P1 > 1 ? 1 : 0] = v.y;
     }
 #pragma unroll
-    for (int gi = 0; gi < 8; ++gi) {
+    for (int gi = 0; gi < 4; ++gi) {
         uint32_t o[4];
         if (P0 == 4) {
             ext4(d[gi], k[0], k[1], o);
@@ -185,17 +204,12 @@ __device__ __forceinline__ void dequant_row_half(const uint8_t* payload, const _
         } else if (P0 == 2) {
             ext2(d[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, k, o);
         } else {
-            const int bi = gi & 3;
-            ext1(d[gi >> 2], bi | (4 << 4) | (bi << 8) | (4 << 12), k, o);
+            ext1(d[0], gi | (4 << 4) | (gi << 8) | (4 << 12), k, o);
         }
         if (P1 > 0) {
             uint32_t h[4];
-            if (P1 == 1) {
-                const int bi = gi & 3;
-                ext1_hi<P0>(e[gi >> 2], bi | (4 << 4) | (bi << 8) | (4 << 12), h);
-            } else {
-                ext2_hi(e[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, h);
-            }
+            if (P1 == 1) ext1_hi<P0>(e[0], gi | (4 << 4) | (gi << 8) | (4 << 12), h);
+            else ext2_hi(e[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, h);
 #pragma unroll
             for (int j = 0; j < 4; ++j) o[j] = h2_bits(__hadd2(bits_h2(o[j]), bits_h2(h[j])));
         }
@@ -214,8 +228,9 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     // the next kernel may launch once every CTA of this grid has started; it
     // waits (griddepcontrol.wait) for this grid before touching its memory
     pdl_launch_dependents();
-    // the operand tiles need 1024-byte alignment (128B swizzle atoms)
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // the operand tiles need 1024-byte alignment (128B swizzle atoms); pointer
+    // arithmetic on smem_raw keeps the shared address space for the compiler
+    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(base);
     uint32_t* tab = reinterpret_cast<uint32_t*>(base + sizeof(PrefillSmem));  // [2][KB][3]
 
@@ -238,9 +253,13 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         tab[3 * i] = co; tab[3 * i + 1] = so; tab[3 * i + 2] = bits;
     }
     if (tid == 0) {
-        for (int s = 0; s < PF_AB_STAGES; ++s) {
-            mbar_init(&S.full_ab[s], 1 + PF_DQ_WARPS);
-            mbar_init(&S.empty_ab[s], 1);
+        for (int s = 0; s < PF_A_STAGES; ++s) {
+            mbar_init(&S.full_a[s], PF_DQ_WARPS);
+            mbar_init(&S.empty_a[s], 1);
+        }
+        for (int s = 0; s < PF_B_STAGES; ++s) {
+            mbar_init(&S.full_b[s], 1);
+            mbar_init(&S.empty_b[s], 1);
         }
         for (int s = 0; s < PF_C_STAGES; ++s) {
             mbar_init(&S.full_c[s], 1);
@@ -269,8 +288,9 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     auto bits_of = [&](int h, int kb) -> uint32_t { return tab[3 * (h * KB + kb) + 2]; };
 
     if (warp == 0) {
-        // ------------------------------ producer ------------------------------
-        pdl_wait();   // x' and tok_scale come from the prologue kernel
+        // -------------------- producer of the packed codes --------------------
+        // runs as far ahead as the code stages allow (the weights do not
+        // depend on the prologue kernel)
         if (lane == 0) {
             int a = 0;
             for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
@@ -290,12 +310,22 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                     bulk_g2s(cst + 16384 + h * 256, p.scales + so, 128u, &S.full_c[sc]);
                     bulk_g2s(cst + 16384 + h * 256 + 128, p.zeros + so, 128u, &S.full_c[sc]);
                 }
-                const int s = a % PF_AB_STAGES;
-                const uint32_t ps = (uint32_t)(a / PF_AB_STAGES) & 1u;
-                if (!mbar_wait_bounded(&S.empty_ab[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
-                mbar_arrive_expect_tx(&S.full_ab[s], (uint32_t)PF_B_BYTES);
-                tma_load_2d(S.b[s], &tmap_x, kb * 128, m0, &S.full_ab[s]);
-                tma_load_2d(S.b[s] + PF_BN * 128, &tmap_x, kb * 128 + 64, m0, &S.full_ab[s]);
+                ++a;
+            }
+        }
+    } else if (warp == PF_WARPS - 1) {
+        // ------------------- producer of the activation tiles -----------------
+        pdl_wait();   // x' comes from the prologue kernel
+        if (lane == 0) {
+            int a = 0;
+            for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
+                if ((bits_of(0, kb) | bits_of(1, kb)) == 0) continue;
+                const int s = a % PF_B_STAGES;
+                const uint32_t ps = (uint32_t)(a / PF_B_STAGES) & 1u;
+                if (!mbar_wait_bounded(&S.empty_b[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
+                mbar_arrive_expect_tx(&S.full_b[s], (uint32_t)PF_B_BYTES);
+                tma_load_2d(S.b[s], &tmap_x, kb * 128, m0, &S.full_b[s]);
+                tma_load_2d(S.b[s] + PF_BN * 128, &tmap_x, kb * 128 + 64, m0, &S.full_b[s]);
                 ++a;
             }
         }
@@ -306,11 +336,12 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         if (lane == 0) {
             for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
                 if ((bits_of(0, kb) | bits_of(1, kb)) == 0) continue;
-                const int s = a % PF_AB_STAGES;
-                const uint32_t ps = (uint32_t)(a / PF_AB_STAGES) & 1u;
-                if (!mbar_wait_bounded(&S.full_ab[s], ps, DEC_WAIT_NS)) { timed_out(); break; }
+                const int sa = a % PF_A_STAGES, sb = a % PF_B_STAGES;
+                const uint32_t pa = (uint32_t)(a / PF_A_STAGES) & 1u, pb = (uint32_t)(a / PF_B_STAGES) & 1u;
+                if (!mbar_wait_bounded(&S.full_a[sa], pa, DEC_WAIT_NS)) { timed_out(); break; }
+                if (!mbar_wait_bounded(&S.full_b[sb], pb, DEC_WAIT_NS)) { timed_out(); break; }
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(S.a[s]), b_base = smem_u32(S.b[s]);
+                const uint32_t a_base = smem_u32(S.a[sa]), b_base = smem_u32(S.b[sb]);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * (PF_BM * 128) + (kk & 3) * 32);
@@ -319,7 +350,8 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                                 umma_smem_desc_sw128(b_base + offb), idesc,
                                 (a > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&S.empty_ab[s]);
+                umma_commit(&S.empty_a[sa]);
+                umma_commit(&S.empty_b[sb]);
                 ++a;
             }
             if (a > 0) umma_commit(&S.d_full);
@@ -328,11 +360,14 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         __syncwarp();
     } else {
         // ---------------------- dequantize, then epilogue ----------------------
-        const int dw = warp - 2;                 // 0..7
-        const int quad = warp & 3;               // TMEM lane quadrant of this warp
-        const int half = dw >> 2;                // which 64 K / 64 tokens this warp takes
-        const int r = quad * 32 + lane;          // weight row in the tile (= TMEM lane)
+        const int dw = warp - 2;                 // 0..15
+        // dequantization: rows 8*dw .. 8*dw+7, lane = row * 4 + quarter
+        const int r = 8 * dw + (lane >> 2);
         const int h = r >> 6, rr = r & 63;
+        const int g0 = 4 * (lane & 3);           // the quarter's first group of 8 codes
+        // epilogue: TMEM lane quadrant of this warp, and which 32 tokens it takes
+        const int quad = warp & 3;
+        const int part = dw >> 2;
         int a = 0;
         bool any = false;
         for (int kb = 0; kb < KB; ++kb) {
@@ -342,50 +377,53 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
             if (S.abort_flag) break;
             const int sc = a % PF_C_STAGES;
             const uint32_t pc = (uint32_t)(a / PF_C_STAGES) & 1u;
-            const int s = a % PF_AB_STAGES;
-            const uint32_t ps = (uint32_t)(a / PF_AB_STAGES) & 1u;
+            const int s = a % PF_A_STAGES;
+            const uint32_t ps = (uint32_t)(a / PF_A_STAGES) & 1u;
             bool ok = mbar_wait_bounded(&S.full_c[sc], pc, DEC_WAIT_NS);
-            ok = ok && mbar_wait_bounded(&S.empty_ab[s], ps ^ 1u, DEC_WAIT_NS);
+            ok = ok && mbar_wait_bounded(&S.empty_a[s], ps ^ 1u, DEC_WAIT_NS);
             if (!__all_sync(0xffffffffu, ok)) { if (lane == 0) timed_out(); break; }
             const uint32_t b = h ? b1 : b0;
             uint8_t* a_tile = S.a[s];
             const uint8_t* cst = S.c[sc];
             const __half* scz = reinterpret_cast<const __half*>(cst + 16384 + h * 256);
-            const int g0 = half * 8;
             switch (b) {
                 case 0: {
                     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int gi = 0; gi < 8; ++gi)
+                    for (int gi = 0; gi < 4; ++gi)
                         *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + gi)) = zero;
                     break;
                 }
-                case 1: dequant_row_half<1>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
-                case 2: dequant_row_half<2>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
-                case 3: dequant_row_half<3>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
-                case 4: dequant_row_half<4>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
-                case 5: dequant_row_half<5>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
-                case 6: dequant_row_half<6>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
-                default: dequant_row_half<8>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 1: dequant_row_part<1>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 2: dequant_row_part<2>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 3: dequant_row_part<3>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 4: dequant_row_part<4>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 5: dequant_row_part<5>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                case 6: dequant_row_part<6>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
+                default: dequant_row_part<8>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
             }
             fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&S.full_ab[s]);
+                mbar_arrive(&S.full_a[s]);
                 mbar_arrive(&S.empty_c[sc]);
             }
             ++a;
         }
-        // epilogue: this warp's 32 rows x its 64 tokens
+        // epilogue: this warp's 32 rows x its 32 tokens
         pdl_wait();   // tok_scale comes from the prologue kernel
         bool ok = S.abort_flag ? false : mbar_wait_bounded(&S.d_full, 0u, DEC_WAIT_NS);
-        if (!__all_sync(0xffffffffu, ok) && !S.abort_flag && lane == 0) timed_out();
+        ok = __all_sync(0xffffffffu, ok);   // warp-uniform: tcgen05.ld is .sync.aligned
+        if (!ok && !S.abort_flag && lane == 0) timed_out();
         tc_fence_after();
-        const int i = nb0 * 64 + r;
+        const int re = quad * 32 + lane;         // TMEM lane = weight row of the tile
+        const int i = nb0 * 64 + re;
         const bool row_ok = i < p.N;
-        const int n = row_ok ? (p.row_perm ? p.row_perm[i] : i) : 0;
-        for (int cc = 0; cc < 2; ++cc) {
-            const int col0 = half * 64 + cc * 32;
+        // in W' row order the 32 lanes write 32 consecutive floats (one 128-byte
+        // line); through row_perm every value would be a separate scattered store
+        const int n = row_ok ? ((p.row_perm && !p.permuted_out) ? p.row_perm[i] : i) : 0;
+        {
+            const int col0 = part * 32;
             float v[32];
             if (any && ok) {
                 tmem_ld32(tmem_d + ((uint32_t)(quad * 32) << 16) + (uint32_t)col0, v);
@@ -410,6 +448,24 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                      "r"(PF_TMEM_COLS)
                      : "memory");
     }
+}
+
+// ---------------------------------------------------------------------------
+// Inverse output reordering after the tensor-core kernel: y[m][row_perm[i]] =
+// y'[m][i], in place.  One CTA per token row: the row is read coalesced and
+// scattered into shared memory through row_perm, then written back coalesced.
+// (SFMP abstract: the reordering costs only a small reordering step.)
+// ---------------------------------------------------------------------------
+constexpr int UNPERM_THREADS = 512;
+
+__global__ void __launch_bounds__(UNPERM_THREADS) k_unpermute_rows(float* y, const int32_t* row_perm, int N) {
+    extern __shared__ float srow[];
+    pdl_launch_dependents();
+    pdl_wait();   // y' comes from the kernel before
+    float* yr = y + (size_t)blockIdx.x * N;
+    for (int i = threadIdx.x; i < N; i += UNPERM_THREADS) srow[row_perm[i]] = yr[i];
+    __syncthreads();
+    for (int n = threadIdx.x; n < N; n += UNPERM_THREADS) yr[n] = srow[n];
 }
 
 }  // namespace mpq

@@ -221,6 +221,8 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
 std::atomic<uint64_t> g_decode_attr{0};
 std::atomic<uint64_t> g_decode_attr8{0};
 std::atomic<uint64_t> g_prefill_attr{0};
+std::atomic<uint64_t> g_unperm_attr{0};
+constexpr size_t kUnpermMaxBytes = 200 * 1024;   // one row of y in shared memory
 
 // cuTensorMapEncodeTiled from the driver, looked up through the runtime.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -419,6 +421,13 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         pp.KB = KB;
         pp.M = M;
         pp.tiles_n = (NB + 1) / 2;
+        // W'-order output + an in-place reordering kernel when a row of y fits
+        // in shared memory; otherwise the epilogue scatters through row_perm
+        pp.permuted_out = (layer->row_perm && (size_t)layer->N * 4 <= kUnpermMaxBytes) ? 1 : 0;
+        if (pp.permuted_out) {
+            e = ensure_smem_attr(k_unpermute_rows, (int)kUnpermMaxBytes, g_unperm_attr);
+            if (e != cudaSuccess) return MPQ_ERR_CUDA;
+        }
         const int tiles_m = (M + PF_BN - 1) / PF_BN;
         cudaLaunchConfig_t pc{};
         pc.gridDim = dim3((unsigned)(pp.tiles_n * tiles_m));
@@ -431,6 +440,17 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
             return MPQ_ERR_CUDA;
         e = cudaLaunchKernelEx(&pc, k_prefill, pp, tmap);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
+        if (pp.permuted_out) {
+            cudaLaunchConfig_t uc{};
+            uc.gridDim = dim3((unsigned)M);
+            uc.blockDim = dim3(UNPERM_THREADS);
+            uc.dynamicSmemBytes = (size_t)layer->N * 4;
+            uc.stream = s;
+            uc.attrs = pdl;
+            uc.numAttrs = 1;
+            e = cudaLaunchKernelEx(&uc, k_unpermute_rows, y_dev, layer->row_perm, layer->N);
+            if (e != cudaSuccess) return MPQ_ERR_CUDA;
+        }
         if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
             return MPQ_ERR_CUDA;
         return MPQ_OK;
