@@ -83,11 +83,23 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
     std::vector<uint32_t> bounds;
     bounds.reserve((size_t)want + 1);
     bounds.push_back(0u);
-    for (int64_t u = 1; u < want; ++u) {
-        // run u starts at the first block whose cost prefix reaches u*cost/want
-        const uint64_t target = (uint64_t)((unsigned __int128)u * cost / (uint64_t)want);
-        const uint32_t tb = (uint32_t)(std::lower_bound(pre.begin(), pre.begin() + T, target) - pre.begin());
-        if (tb > bounds.back() && tb < (uint32_t)T) bounds.push_back(tb);
+    if ((uint64_t)want >= nz) {
+        // at least as many runs as non-zero blocks (a small layer): one
+        // non-zero block per run, so that no warp gets two -- zero-bit blocks
+        // join the run before them
+        bool seen_nz = false;
+        for (int64_t t = 0; t < T; ++t) {
+            if (!bits[t]) continue;
+            if (seen_nz) bounds.push_back((uint32_t)t);
+            seen_nz = true;
+        }
+    } else {
+        for (int64_t u = 1; u < want; ++u) {
+            // run u starts at the first block whose cost prefix reaches u*cost/want
+            const uint64_t target = (uint64_t)((unsigned __int128)u * cost / (uint64_t)want);
+            const uint32_t tb = (uint32_t)(std::lower_bound(pre.begin(), pre.begin() + T, target) - pre.begin());
+            if (tb > bounds.back() && tb < (uint32_t)T) bounds.push_back(tb);
+        }
     }
     bounds.push_back((uint32_t)T);
     const int64_t units = (int64_t)bounds.size() - 1;

@@ -27,8 +27,9 @@ def block_cost(b):
 
 
 def restated_schedule(N, K, bits):
-    """The schedule rules, restated: cost-prefix cuts, empty runs dropped,
-    32-word descriptors, then the width byte of every block."""
+    """The schedule rules, restated: cost-prefix cuts (or, when there are no
+    more non-zero blocks than runs, one non-zero block per run), empty runs
+    dropped, 32-word descriptors, then the width byte of every block."""
     NB, KB = N // 64, K // 128
     T = NB * KB
     bits = np.asarray(bits, np.int64)
@@ -37,11 +38,15 @@ def restated_schedule(N, K, bits):
     total = int(pre[-1])
     want = max(1, min(-(-total // MIN_UNIT_COST), MAX_UNITS, T))
     bounds = [0]
-    for u in range(1, want):
-        tgt = u * total // want
-        tb = int(np.searchsorted(pre[:T], tgt, side="left"))
-        if bounds[-1] < tb < T:
-            bounds.append(tb)
+    nz = np.flatnonzero(bits)
+    if want >= len(nz):            # small layer: one non-zero block per run
+        bounds += [int(t) for t in nz[1:]]
+    else:
+        for u in range(1, want):
+            tgt = u * total // want
+            tb = int(np.searchsorted(pre[:T], tgt, side="left"))
+            if bounds[-1] < tb < T:
+                bounds.append(tb)
     bounds.append(T)
     U = len(bounds) - 1
     row_first = np.zeros(NB, np.int64)
