@@ -302,7 +302,7 @@ __device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
 // Last arriver of a shared block row: y[m][rows[r]] = sum over the row's nc
 // runs (in run order) of their partial sums.  The slots are contiguous
 // ([nc][Mg tokens][64 rows] floats at `slots`); lanes read float4 vectors of
-// them, eight slots per batch with every load of a batch in flight.  With one
+// them, sixteen slots per batch with every load of a batch in flight.  With one
 // token a slot is 16 vectors, so two lane groups take the even and odd slots
 // and are combined in that order (the sum stays deterministic).  Kept out of
 // line: it runs once per shared row, and its registers must not weigh on the
@@ -315,15 +315,15 @@ __device__ __noinline__ void finish_shared_row(const float* __restrict__ slots, 
     const uint32_t grp = (V == 16u) ? (uint32_t)lane >> 4 : 0u;
     for (uint32_t v = (V == 16u) ? ((uint32_t)lane & 15u) : (uint32_t)lane; v < V; v += 32u) {
         float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (uint32_t c0 = grp; c0 < nc; c0 += 8u * groups) {
-            float4 q[8];
+        for (uint32_t c0 = grp; c0 < nc; c0 += 16u * groups) {
+            float4 q[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 16; ++k) {
                 const uint32_t c = c0 + (uint32_t)k * groups;
                 q[k] = c < nc ? __ldcg(pv + (size_t)c * V + v) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 16; ++k) {
                 tot.x += q[k].x; tot.y += q[k].y; tot.z += q[k].z; tot.w += q[k].w;
             }
         }

@@ -162,35 +162,30 @@ constexpr int XPREP_DEC_WARPS = XPREP_THREADS / 32;
 
 __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
     pdl_launch_dependents();
-    pdl_wait();   // the kernel before may still read the workspace or write x
     __shared__ float xs[XPREP_DEC_WARPS][64];   // 128 fp16 per warp
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int KB = p.K / 128;
+    const int item = blockIdx.x * XPREP_DEC_WARPS + warp;   // = kb * M + m
+    const bool active = item < KB * p.M;
+    const int kb = active ? item / p.M : 0, m = active ? item % p.M : 0;
+    // lane holds columns 4*lane .. 4*lane+3 of the slice; the column order is
+    // static, so it is read before waiting for the kernel that writes x
+    const int c0 = kb * 128 + 4 * lane;
+    int4 cp = make_int4(c0, c0 + 1, c0 + 2, c0 + 3);
+    if (p.col_perm && active) cp = *reinterpret_cast<const int4*>(p.col_perm + c0);
+    pdl_wait();   // the kernel before may still read the workspace or write x
     if (blockIdx.x == 0) {
         if (tid == 0 && p.err) *p.err = 0u;
         if (p.counters)
             for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
     }
-    const int item = blockIdx.x * XPREP_DEC_WARPS + warp;   // = kb * M + m
-    if (item >= KB * p.M) return;
-    const int kb = item / p.M, m = item % p.M;
+    if (!active) return;
     const uint16_t* xr = p.x + (size_t)m * p.K;
-    // lane holds columns 4*lane .. 4*lane+3 of the slice
     float v[4];
-    const int c0 = kb * 128 + 4 * lane;
-    if (p.col_perm) {
-        const int4 cp = *reinterpret_cast<const int4*>(p.col_perm + c0);
-        v[0] = __uint_as_float((uint32_t)xr[cp.x] << 16);
-        v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
-        v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
-        v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
-    } else {
-        const uint2 raw = *reinterpret_cast<const uint2*>(xr + c0);
-        v[0] = __uint_as_float(raw.x << 16);
-        v[1] = __uint_as_float(raw.x & 0xffff0000u);
-        v[2] = __uint_as_float(raw.y << 16);
-        v[3] = __uint_as_float(raw.y & 0xffff0000u);
-    }
+    v[0] = __uint_as_float((uint32_t)xr[cp.x] << 16);
+    v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
+    v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
+    v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
     float amax = 0.f;
 #pragma unroll
     for (int e4 = 0; e4 < 4; ++e4) {
