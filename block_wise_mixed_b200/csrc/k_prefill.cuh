@@ -44,25 +44,32 @@ constexpr int PF_DQ_WARPS = 16;                  // warps 2 .. 17
 constexpr int PF_WARPS = PF_DQ_WARPS + 3;
 constexpr int PF_THREADS = PF_WARPS * 32;
 constexpr int PF_BM = 128;       // weight rows per tile (2 block rows)
-constexpr int PF_BN = 128;       // tokens per tile
 constexpr int PF_A_STAGES = 2;   // dequantized weight tiles
-constexpr int PF_B_STAGES = 2;   // activation tiles (from L2)
-constexpr int PF_C_STAGES = 5;   // packed codes (from HBM: the longer latency)
 constexpr int PF_A_BYTES = PF_BM * 256;           // 128 rows x 128 fp16
-constexpr int PF_B_BYTES = PF_BN * 256;           // 128 tokens x 128 fp16
 constexpr int PF_C_BYTES = 2 * 8192 + 4 * 128;    // two payloads + 2 x (scales, zeros)
-constexpr uint32_t PF_TMEM_COLS = 128;
 
+// Tokens per tile: 128, or 256 for large batches (each dequantized weight
+// tile then feeds twice the tensor-core work).  Activation stages hold half
+// a k block (64 columns) so that both fit in shared memory.
+template <int BN>
+struct PfCfg {
+    static constexpr int B_STAGES = BN == 256 ? 3 : 4;   // half-k-block activation stages (from L2)
+    static constexpr int B_BYTES = BN * 128;              // BN tokens x 64 fp16
+    static constexpr int C_STAGES = BN == 256 ? 3 : 5;   // packed codes (from HBM)
+    static constexpr uint32_t TMEM_COLS = BN;             // fp32 accumulator columns
+};
+
+template <int BN>
 struct PrefillSmem {
     uint8_t a[PF_A_STAGES][PF_A_BYTES];    // 1024-aligned (offset 0)
-    uint8_t b[PF_B_STAGES][PF_B_BYTES];
-    uint8_t c[PF_C_STAGES][PF_C_BYTES];
+    uint8_t b[PfCfg<BN>::B_STAGES][PfCfg<BN>::B_BYTES];
+    uint8_t c[PfCfg<BN>::C_STAGES][PF_C_BYTES];
     uint64_t full_a[PF_A_STAGES];
     uint64_t empty_a[PF_A_STAGES];
-    uint64_t full_b[PF_B_STAGES];
-    uint64_t empty_b[PF_B_STAGES];
-    uint64_t full_c[PF_C_STAGES];
-    uint64_t empty_c[PF_C_STAGES];
+    uint64_t full_b[PfCfg<BN>::B_STAGES];
+    uint64_t empty_b[PfCfg<BN>::B_STAGES];
+    uint64_t full_c[PfCfg<BN>::C_STAGES];
+    uint64_t empty_c[PfCfg<BN>::C_STAGES];
     uint64_t d_full;
     uint32_t tmem_base;
     volatile int abort_flag;
@@ -222,8 +229,12 @@ __device__ __forceinline__ void dequant_row_part(const uint8_t* payload, const _
     }
 }
 
+template <int BN>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
+    using Cfg = PfCfg<BN>;
+    constexpr int PF_C_STAGES = Cfg::C_STAGES;
+    constexpr int PF_B_STAGES = Cfg::B_STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the next kernel may launch once every CTA of this grid has started; it
     // waits (griddepcontrol.wait) for this grid before touching its memory
@@ -231,15 +242,15 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     // the operand tiles need 1024-byte alignment (128B swizzle atoms); pointer
     // arithmetic on smem_raw keeps the shared address space for the compiler
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(base);
-    uint32_t* tab = reinterpret_cast<uint32_t*>(base + sizeof(PrefillSmem));  // [2][KB][3]
+    PrefillSmem<BN>& S = *reinterpret_cast<PrefillSmem<BN>*>(base);
+    uint32_t* tab = reinterpret_cast<uint32_t*>(base + sizeof(PrefillSmem<BN>));  // [2][KB][3]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int KB = p.KB;
     const int tile_n = blockIdx.x % p.tiles_n;
     const int tile_m = blockIdx.x / p.tiles_n;
     const int nb0 = 2 * tile_n;
-    const int m0 = tile_m * PF_BN;
+    const int m0 = tile_m * BN;
 
     // stage this tile's table entries: tab[(h*KB + kb)*3 + {0,1,2}]
     for (int i = tid; i < 2 * KB; i += PF_THREADS) {
@@ -272,7 +283,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&S.tmem_base)),
-                     "r"(PF_TMEM_COLS)
+                     "r"(Cfg::TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -317,41 +328,49 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         // ------------------- producer of the activation tiles -----------------
         pdl_wait();   // x' comes from the prologue kernel
         if (lane == 0) {
-            int a = 0;
+            int bq = 0;   // half-k-block activation tiles issued
             for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
                 if ((bits_of(0, kb) | bits_of(1, kb)) == 0) continue;
-                const int s = a % PF_B_STAGES;
-                const uint32_t ps = (uint32_t)(a / PF_B_STAGES) & 1u;
-                if (!mbar_wait_bounded(&S.empty_b[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
-                mbar_arrive_expect_tx(&S.full_b[s], (uint32_t)PF_B_BYTES);
-                tma_load_2d(S.b[s], &tmap_x, kb * 128, m0, &S.full_b[s]);
-                tma_load_2d(S.b[s] + PF_BN * 128, &tmap_x, kb * 128 + 64, m0, &S.full_b[s]);
-                ++a;
+                for (int hh = 0; hh < 2; ++hh, ++bq) {
+                    const int s = bq % PF_B_STAGES;
+                    const uint32_t ps = (uint32_t)(bq / PF_B_STAGES) & 1u;
+                    if (!mbar_wait_bounded(&S.empty_b[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
+                    mbar_arrive_expect_tx(&S.full_b[s], (uint32_t)Cfg::B_BYTES);
+                    tma_load_2d(S.b[s], &tmap_x, kb * 128 + 64 * hh, m0, &S.full_b[s]);
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ----------------------------
-        const uint32_t idesc = umma_idesc_f16(PF_BM, PF_BN);
+        const uint32_t idesc = umma_idesc_f16(PF_BM, BN);
         int a = 0;
         if (lane == 0) {
-            for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
+            bool stop = false;
+            for (int kb = 0; kb < KB && !S.abort_flag && !stop; ++kb) {
                 if ((bits_of(0, kb) | bits_of(1, kb)) == 0) continue;
-                const int sa = a % PF_A_STAGES, sb = a % PF_B_STAGES;
-                const uint32_t pa = (uint32_t)(a / PF_A_STAGES) & 1u, pb = (uint32_t)(a / PF_B_STAGES) & 1u;
+                const int sa = a % PF_A_STAGES;
+                const uint32_t pa = (uint32_t)(a / PF_A_STAGES) & 1u;
                 if (!mbar_wait_bounded(&S.full_a[sa], pa, DEC_WAIT_NS)) { timed_out(); break; }
-                if (!mbar_wait_bounded(&S.full_b[sb], pb, DEC_WAIT_NS)) { timed_out(); break; }
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(S.a[sa]), b_base = smem_u32(S.b[sb]);
+                const uint32_t a_base = smem_u32(S.a[sa]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int bq = 2 * a + hh;
+                    const int sb = bq % PF_B_STAGES;
+                    const uint32_t pb = (uint32_t)(bq / PF_B_STAGES) & 1u;
+                    if (!mbar_wait_bounded(&S.full_b[sb], pb, DEC_WAIT_NS)) { timed_out(); stop = true; break; }
+                    tc_fence_after();
+                    const uint32_t b_base = smem_u32(S.b[sb]);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * (PF_BM * 128) + (kk & 3) * 32);
-                    const uint32_t offb = (uint32_t)((kk >> 2) * (PF_BN * 128) + (kk & 3) * 32);
-                    umma_f16_ss(tmem_d, umma_smem_desc_sw128(a_base + off),
-                                umma_smem_desc_sw128(b_base + offb), idesc,
-                                (a > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // A: the 64-column half hh of the k block; B: this half's stage
+                        const uint32_t off = (uint32_t)(hh * (PF_BM * 128) + kk * 32);
+                        umma_f16_ss(tmem_d, umma_smem_desc_sw128(a_base + off),
+                                    umma_smem_desc_sw128(b_base + (uint32_t)(kk * 32)), idesc,
+                                    (a > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&S.empty_b[sb]);
                 }
+                if (stop) break;
                 umma_commit(&S.empty_a[sa]);
-                umma_commit(&S.empty_b[sb]);
                 ++a;
             }
             if (a > 0) umma_commit(&S.d_full);
@@ -410,7 +429,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
             }
             ++a;
         }
-        // epilogue: this warp's 32 rows x its 32 tokens
+        // epilogue: this warp's 32 rows x its BN/4 tokens
         pdl_wait();   // tok_scale comes from the prologue kernel
         bool ok = S.abort_flag ? false : mbar_wait_bounded(&S.d_full, 0u, DEC_WAIT_NS);
         ok = __all_sync(0xffffffffu, ok);   // warp-uniform: tcgen05.ld is .sync.aligned
@@ -422,8 +441,8 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         // in W' row order the 32 lanes write 32 consecutive floats (one 128-byte
         // line); through row_perm every value would be a separate scattered store
         const int n = row_ok ? ((p.row_perm && !p.permuted_out) ? p.row_perm[i] : i) : 0;
-        {
-            const int col0 = part * 32;
+        for (int cc = 0; cc < BN / 128; ++cc) {
+            const int col0 = part * (BN / 4) + cc * 32;
             float v[32];
             if (any && ok) {
                 tmem_ld32(tmem_d + ((uint32_t)(quad * 32) << 16) + (uint32_t)col0, v);
@@ -445,7 +464,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d),
-                     "r"(PF_TMEM_COLS)
+                     "r"(Cfg::TMEM_COLS)
                      : "memory");
     }
 }

@@ -233,6 +233,7 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
 std::atomic<uint64_t> g_decode_attr{0};
 std::atomic<uint64_t> g_decode_attr8{0};
 std::atomic<uint64_t> g_prefill_attr{0};
+std::atomic<uint64_t> g_prefill_attr256{0};
 std::atomic<uint64_t> g_unperm_attr{0};
 constexpr size_t kUnpermMaxBytes = 200 * 1024;   // one row of y in shared memory
 
@@ -263,9 +264,12 @@ bool make_tmap_fp16(CUtensorMap* map, const void* ptr, int K, int rows, int box_
     return r == CUDA_SUCCESS;
 }
 
+template <int BN>
 size_t prefill_smem_bytes(int KB) {
-    return sizeof(PrefillSmem) + 1024 + (size_t)2 * KB * 12;
+    return sizeof(PrefillSmem<BN>) + 1024 + (size_t)2 * KB * 12;
 }
+// 256-token tiles once there are enough of them to fill the SMs
+constexpr int kPrefillWideM = 1024;
 
 }  // namespace
 
@@ -412,12 +416,15 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
 
     if (use_tc) {
-        const size_t smem = prefill_smem_bytes(KB);
+        const bool wide = M >= kPrefillWideM;
+        const int BN = wide ? 256 : 128;
+        const size_t smem = wide ? prefill_smem_bytes<256>(KB) : prefill_smem_bytes<128>(KB);
         if (smem > 227 * 1024) return MPQ_ERR_SHAPE;
-        e = ensure_smem_attr(k_prefill, 227 * 1024, g_prefill_attr);   // the sm_100 maximum
+        e = wide ? ensure_smem_attr(k_prefill<256>, 227 * 1024, g_prefill_attr256)   // the sm_100 maximum
+                 : ensure_smem_attr(k_prefill<128>, 227 * 1024, g_prefill_attr);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
         CUtensorMap tmap;
-        if (!make_tmap_fp16(&tmap, w.xq, layer->K, M, PF_BN)) return MPQ_ERR_CUDA;
+        if (!make_tmap_fp16(&tmap, w.xq, layer->K, M, BN)) return MPQ_ERR_CUDA;
         PrefillParams pp{};
         pp.codes = static_cast<const uint8_t*>(layer->codes);
         pp.table = layer->table;
@@ -440,7 +447,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
             e = ensure_smem_attr(k_unpermute_rows, (int)kUnpermMaxBytes, g_unperm_attr);
             if (e != cudaSuccess) return MPQ_ERR_CUDA;
         }
-        const int tiles_m = (M + PF_BN - 1) / PF_BN;
+        const int tiles_m = (M + BN - 1) / BN;
         cudaLaunchConfig_t pc{};
         pc.gridDim = dim3((unsigned)(pp.tiles_n * tiles_m));
         pc.blockDim = dim3(PF_THREADS);
@@ -450,7 +457,8 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         pc.numAttrs = 1;
         if (ev_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s) != cudaSuccess)
             return MPQ_ERR_CUDA;
-        e = cudaLaunchKernelEx(&pc, k_prefill, pp, tmap);
+        e = wide ? cudaLaunchKernelEx(&pc, k_prefill<256>, pp, tmap)
+                 : cudaLaunchKernelEx(&pc, k_prefill<128>, pp, tmap);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
         if (pp.permuted_out) {
             cudaLaunchConfig_t uc{};

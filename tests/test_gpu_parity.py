@@ -214,7 +214,11 @@ def test_linear_host_entry_point(mpq, oracle):
 # sampled output rows the oracle computes one by one.
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("cfg,proj,Ms", [(3, 0, (1, 8, 16, 32)), (3, 2, (1, 8)),
-                                         (4, 1, (1, 4, 16)), (4, 3, (1,))])
+                                         (4, 1, (1, 4, 16)), (4, 3, (1,)),
+                                         # tensor-core path at the prefill sizes: 128-token
+                                         # tiles (512, ragged 700) and 256-token tiles
+                                         # (2048, ragged 1100)
+                                         (5, 0, (512, 2048)), (5, 1, (700,)), (5, 6, (1100,))])
 def test_full_size_sampled(mpq, oracle, cfg, proj, Ms):
     L = synth.config_layer(cfg, proj)
     P = pack_gpu(mpq, L)
