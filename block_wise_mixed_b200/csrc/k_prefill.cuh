@@ -83,11 +83,15 @@ struct PrefillParams {
     const uint16_t* zeros;
     const int32_t* row_perm;
     const float* tok_scale;   // [M]
-    float* y;                 // [M][N]
-    int permuted_out;         // 1: write y in W' row order (k_unpermute_rows fixes it)
+    float* out;               // output base (see out_scatter)
+    int out_scatter;          // 1: out = y, rows scattered through row_perm;
+                              // 0: out = [split][M][N] in W' row order (k_finish_rows
+                              //    adds the splits and applies row_perm)
     uint32_t* err;
     int N, K, NB, KB, M;
     int tiles_n;              // ceil(NB / 2)
+    int tiles_m;              // ceil(M / BN)
+    int kb_per_split;         // k blocks per CTA (split-K when < KB)
 };
 
 __device__ __forceinline__ uint64_t umma_smem_desc_sw128(uint32_t saddr) {
@@ -246,11 +250,15 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     uint32_t* tab = reinterpret_cast<uint32_t*>(base + sizeof(PrefillSmem<BN>));  // [2][KB][3]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int KB = p.KB;
-    const int tile_n = blockIdx.x % p.tiles_n;
-    const int tile_m = blockIdx.x / p.tiles_n;
+    const int tiles = p.tiles_n * p.tiles_m;
+    const int split = blockIdx.x / tiles;
+    const int tile_n = (blockIdx.x % tiles) % p.tiles_n;
+    const int tile_m = (blockIdx.x % tiles) / p.tiles_n;
     const int nb0 = 2 * tile_n;
     const int m0 = tile_m * BN;
+    // this CTA's k blocks: [kb0, kb0 + KB) of the layer's p.KB
+    const int kb0 = split * p.kb_per_split;
+    const int KB = max(0, min(p.KB, kb0 + p.kb_per_split) - kb0);
 
     // stage this tile's table entries: tab[(h*KB + kb)*3 + {0,1,2}]
     for (int i = tid; i < 2 * KB; i += PF_THREADS) {
@@ -258,7 +266,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         const int nb = nb0 + h;
         uint32_t co = 0, so = 0, bits = 0;
         if (nb < p.NB) {
-            const mpq_block e = p.table[(size_t)nb * KB + kb];
+            const mpq_block e = p.table[(size_t)nb * p.KB + kb0 + kb];
             co = e.code_off; so = e.sz_off; bits = e.bits;
         }
         tab[3 * i] = co; tab[3 * i + 1] = so; tab[3 * i + 2] = bits;
@@ -336,7 +344,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                     const uint32_t ps = (uint32_t)(bq / PF_B_STAGES) & 1u;
                     if (!mbar_wait_bounded(&S.empty_b[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
                     mbar_arrive_expect_tx(&S.full_b[s], (uint32_t)Cfg::B_BYTES);
-                    tma_load_2d(S.b[s], &tmap_x, kb * 128 + 64 * hh, m0, &S.full_b[s]);
+                    tma_load_2d(S.b[s], &tmap_x, (kb0 + kb) * 128 + 64 * hh, m0, &S.full_b[s]);
                 }
             }
         }
@@ -440,7 +448,8 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         const bool row_ok = i < p.N;
         // in W' row order the 32 lanes write 32 consecutive floats (one 128-byte
         // line); through row_perm every value would be a separate scattered store
-        const int n = row_ok ? ((p.row_perm && !p.permuted_out) ? p.row_perm[i] : i) : 0;
+        const int n = row_ok ? ((p.row_perm && p.out_scatter) ? p.row_perm[i] : i) : 0;
+        float* out = p.out + (p.out_scatter ? 0 : (size_t)split * p.M * p.N);
         for (int cc = 0; cc < BN / 128; ++cc) {
             const int col0 = part * (BN / 4) + cc * 32;
             float v[32];
@@ -454,7 +463,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int m = m0 + col0 + j;
-                    if (m < p.M) p.y[(size_t)m * p.N + n] = v[j] * p.tok_scale[m];
+                    if (m < p.M) out[(size_t)m * p.N + n] = v[j] * p.tok_scale[m];
                 }
             }
         }
@@ -470,21 +479,79 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
 }
 
 // ---------------------------------------------------------------------------
-// Inverse output reordering after the tensor-core kernel: y[m][row_perm[i]] =
-// y'[m][i], in place.  One CTA per token row: the row is read coalesced and
-// scattered into shared memory through row_perm, then written back coalesced.
-// (SFMP abstract: the reordering costs only a small reordering step.)
+// After the tensor-core kernel: y[m][row_perm[i]] = sum over the k splits (in
+// split order) of part[split][m][i].  One CTA per token row: the splits' rows
+// are read coalesced and their sum scattered into shared memory through
+// row_perm, then the row is written back coalesced.  part may be y itself
+// (one split: the reordering is then in place; every thread reads before any
+// writes, after the barrier).  (SFMP abstract: the reordering costs only a
+// small step.)
 // ---------------------------------------------------------------------------
-constexpr int UNPERM_THREADS = 512;
+constexpr int FINISH_THREADS = 512;
 
-__global__ void __launch_bounds__(UNPERM_THREADS) k_unpermute_rows(float* y, const int32_t* row_perm, int N) {
-    extern __shared__ float srow[];
+__device__ __forceinline__ void f4_acc(float4& a, const float4 b) {
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+}
+
+// The sum over the splits of four consecutive values of a row, stored as
+// mode says: 0 at their own columns, 1 into shared memory through row_perm,
+// 2 straight to y through row_perm.
+__device__ __forceinline__ void finish_put4(float* yr, float* srow, const int32_t* row_perm, int i4,
+                                            float4 v, int mode) {
+    if (mode == 0) {
+        reinterpret_cast<float4*>(yr)[i4] = v;
+        return;
+    }
+    const int4 r = reinterpret_cast<const int4*>(row_perm)[i4];
+    float* dst = mode == 1 ? srow : yr;
+    dst[r.x] = v.x; dst[r.y] = v.y; dst[r.z] = v.z; dst[r.w] = v.w;
+}
+
+__global__ void __launch_bounds__(FINISH_THREADS) k_finish_rows(float* y, const float* part, int splits,
+                                                               size_t split_stride, const int32_t* row_perm,
+                                                               int N, int mode) {
+    // mode 0: no row order; 1: reorder through shared memory; 2: scattered
+    // stores (a row of y larger than shared memory)
+    extern __shared__ __align__(16) float srow[];
     pdl_launch_dependents();
-    pdl_wait();   // y' comes from the kernel before
-    float* yr = y + (size_t)blockIdx.x * N;
-    for (int i = threadIdx.x; i < N; i += UNPERM_THREADS) srow[row_perm[i]] = yr[i];
+    pdl_wait();   // the partial sums come from the kernel before
+    const size_t row = (size_t)blockIdx.x * N;
+    float* yr = y + row;
+    const float* pr = part + row;
+    const bool vec = (N % 4 == 0) && (split_stride % 4 == 0) &&
+                     (((uintptr_t)yr | (uintptr_t)pr | (uintptr_t)row_perm) & 15) == 0;
+    if (vec) {
+        // 16-byte loads, two of them in flight per thread and split
+        const int n4 = N / 4;
+        for (int i0 = threadIdx.x; i0 < n4; i0 += 2 * FINISH_THREADS) {
+            const int i1 = i0 + FINISH_THREADS;
+            const bool two = i1 < n4;
+            float4 a = reinterpret_cast<const float4*>(pr)[i0];
+            float4 b = two ? reinterpret_cast<const float4*>(pr)[i1] : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int sp = 1; sp < splits; ++sp) {
+                const float4* ps = reinterpret_cast<const float4*>(pr + (size_t)sp * split_stride);
+                f4_acc(a, ps[i0]);
+                if (two) f4_acc(b, ps[i1]);
+            }
+            finish_put4(yr, srow, row_perm, i0, a, mode);
+            if (two) finish_put4(yr, srow, row_perm, i1, b, mode);
+        }
+    } else {
+        for (int i = threadIdx.x; i < N; i += FINISH_THREADS) {
+            float v = pr[i];
+            for (int sp = 1; sp < splits; ++sp) v += pr[(size_t)sp * split_stride + i];
+            if (mode == 0) yr[i] = v;
+            else (mode == 1 ? srow : yr)[row_perm[i]] = v;
+        }
+    }
+    if (mode != 1) return;
     __syncthreads();
-    for (int n = threadIdx.x; n < N; n += UNPERM_THREADS) yr[n] = srow[n];
+    if (vec) {
+        for (int i4 = threadIdx.x; i4 < N / 4; i4 += FINISH_THREADS)
+            reinterpret_cast<float4*>(yr)[i4] = reinterpret_cast<const float4*>(srow)[i4];
+    } else {
+        for (int n = threadIdx.x; n < N; n += FINISH_THREADS) yr[n] = srow[n];
+    }
 }
 
 }  // namespace mpq

@@ -180,6 +180,26 @@ bool perm_ok(const int32_t* p, int n) {
 
 inline mpq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MPQ_OK : MPQ_ERR_CUDA; }
 
+// Tensor-core launch shape: 256-token tiles beyond one 128-token tile, and
+// the k blocks split across CTAs (partial sums reduced by k_finish_rows)
+// while the grid stays within one wave of 148 SMs.
+struct PrefillShape {
+    int BN, tiles_n, tiles_m, splits, kb_per_split;
+};
+PrefillShape prefill_shape(int N, int K, int M) {
+    PrefillShape ps{};
+    const int NB = N / 64, KB = K / 128;
+    ps.BN = M > 128 ? 256 : 128;
+    ps.tiles_n = (NB + 1) / 2;
+    ps.tiles_m = (M + ps.BN - 1) / ps.BN;
+    const int ctas = ps.tiles_n * ps.tiles_m;
+    int splits = 1;
+    while (splits < 8 && ctas * splits * 2 <= 148 && KB / (splits * 2) >= 4) splits *= 2;
+    ps.kb_per_split = (KB + splits - 1) / splits;
+    ps.splits = (KB + ps.kb_per_split - 1) / ps.kb_per_split;
+    return ps;
+}
+
 // Workspace carve-up of mpq_linear.
 struct LinearWs {
     uint32_t* err;
@@ -206,7 +226,13 @@ LinearWs carve_linear(void* ws, const mpq_layer* layer, int32_t M) {
     // partial sums of shared block rows: at most n_units + NB slots of
     // 64 rows x (tokens per launch)
     w.partial = reinterpret_cast<float*>(base + off);
-    off += round256((size_t)(layer->n_units + NB) * 64 * std::min(M, kMaxDecodeTokens) * 4);
+    if (M > kDecodeMaxM) {
+        // tensor-core path: [splits][M][N] fp32 partial sums when k is split
+        const PrefillShape ps = prefill_shape(layer->N, layer->K, M);
+        off += round256(ps.splits > 1 ? (size_t)ps.splits * M * layer->N * 4 : 0);
+    } else {
+        off += round256((size_t)(layer->n_units + NB) * 64 * std::min(M, kMaxDecodeTokens) * 4);
+    }
     w.bytes = off;
     return w;
 }
@@ -268,8 +294,7 @@ template <int BN>
 size_t prefill_smem_bytes(int KB) {
     return sizeof(PrefillSmem<BN>) + 1024 + (size_t)2 * KB * 12;
 }
-// 256-token tiles once there are enough of them to fill the SMs
-constexpr int kPrefillWideM = 1024;
+
 
 }  // namespace
 
@@ -416,8 +441,9 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
 
     if (use_tc) {
-        const bool wide = M >= kPrefillWideM;
-        const int BN = wide ? 256 : 128;
+        const PrefillShape shape = prefill_shape(layer->N, layer->K, M);
+        const bool wide = shape.BN == 256;
+        const int BN = shape.BN;
         const size_t smem = wide ? prefill_smem_bytes<256>(KB) : prefill_smem_bytes<128>(KB);
         if (smem > 227 * 1024) return MPQ_ERR_SHAPE;
         e = wide ? ensure_smem_attr(k_prefill<256>, 227 * 1024, g_prefill_attr256)   // the sm_100 maximum
@@ -432,7 +458,8 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         pp.zeros = layer->zeros;
         pp.row_perm = layer->row_perm;
         pp.tok_scale = w.tok_scale;
-        pp.y = y_dev;
+        pp.tiles_m = shape.tiles_m;
+        pp.kb_per_split = shape.kb_per_split;
         pp.err = w.err;
         pp.N = layer->N;
         pp.K = layer->K;
@@ -440,16 +467,21 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         pp.KB = KB;
         pp.M = M;
         pp.tiles_n = (NB + 1) / 2;
-        // W'-order output + an in-place reordering kernel when a row of y fits
-        // in shared memory; otherwise the epilogue scatters through row_perm
-        pp.permuted_out = (layer->row_perm && (size_t)layer->N * 4 <= kUnpermMaxBytes) ? 1 : 0;
-        if (pp.permuted_out) {
-            e = ensure_smem_attr(k_unpermute_rows, (int)kUnpermMaxBytes, g_unperm_attr);
+        // Output: split partials, or y in W' row order reordered in place, go
+        // through k_finish_rows (coalesced stores); the epilogue scatters
+        // through row_perm itself only when a row of y does not fit in shared
+        // memory (and k is not split).
+        const bool row_fits = (size_t)layer->N * 4 <= kUnpermMaxBytes;
+        const bool finish = shape.splits > 1 || (layer->row_perm && row_fits);
+        pp.out_scatter = finish ? 0 : 1;
+        pp.out = shape.splits > 1 ? w.partial : y_dev;
+        if (finish) {
+            e = ensure_smem_attr(k_finish_rows, (int)kUnpermMaxBytes, g_unperm_attr);
             if (e != cudaSuccess) return MPQ_ERR_CUDA;
         }
-        const int tiles_m = (M + BN - 1) / BN;
+        const int tiles_m = shape.tiles_m;
         cudaLaunchConfig_t pc{};
-        pc.gridDim = dim3((unsigned)(pp.tiles_n * tiles_m));
+        pc.gridDim = dim3((unsigned)(pp.tiles_n * tiles_m * shape.splits));
         pc.blockDim = dim3(PF_THREADS);
         pc.dynamicSmemBytes = smem;
         pc.stream = s;
@@ -460,15 +492,18 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         e = wide ? cudaLaunchKernelEx(&pc, k_prefill<256>, pp, tmap)
                  : cudaLaunchKernelEx(&pc, k_prefill<128>, pp, tmap);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
-        if (pp.permuted_out) {
+        if (finish) {
             cudaLaunchConfig_t uc{};
             uc.gridDim = dim3((unsigned)M);
-            uc.blockDim = dim3(UNPERM_THREADS);
-            uc.dynamicSmemBytes = (size_t)layer->N * 4;
+            uc.blockDim = dim3(FINISH_THREADS);
+            // 0: no row order, 1: reorder through shared memory, 2: scattered stores
+            const int mode = !layer->row_perm ? 0 : row_fits ? 1 : 2;
+            uc.dynamicSmemBytes = mode == 1 ? (size_t)layer->N * 4 : 0;
             uc.stream = s;
             uc.attrs = pdl;
             uc.numAttrs = 1;
-            e = cudaLaunchKernelEx(&uc, k_unpermute_rows, y_dev, layer->row_perm, layer->N);
+            e = cudaLaunchKernelEx(&uc, k_finish_rows, y_dev, (const float*)pp.out, shape.splits,
+                                   (size_t)M * layer->N, layer->row_perm, layer->N, mode);
             if (e != cudaSuccess) return MPQ_ERR_CUDA;
         }
         if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
