@@ -493,9 +493,8 @@ __device__ __forceinline__ void f4_acc(float4& a, const float4 b) {
     a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
 }
 
-// The sum over the splits of four consecutive values of a row, stored as
-// mode says: 0 at their own columns, 1 into shared memory through row_perm,
-// 2 straight to y through row_perm.
+// The sum over the splits of four consecutive values of a row, stored at
+// their own columns (mode 0) or into shared memory through row_perm (mode 1).
 __device__ __forceinline__ void finish_put4(float* yr, float* srow, const int32_t* row_perm, int i4,
                                             float4 v, int mode) {
     if (mode == 0) {
@@ -503,15 +502,13 @@ __device__ __forceinline__ void finish_put4(float* yr, float* srow, const int32_
         return;
     }
     const int4 r = reinterpret_cast<const int4*>(row_perm)[i4];
-    float* dst = mode == 1 ? srow : yr;
-    dst[r.x] = v.x; dst[r.y] = v.y; dst[r.z] = v.z; dst[r.w] = v.w;
+    srow[r.x] = v.x; srow[r.y] = v.y; srow[r.z] = v.z; srow[r.w] = v.w;
 }
 
 __global__ void __launch_bounds__(FINISH_THREADS) k_finish_rows(float* y, const float* part, int splits,
                                                                size_t split_stride, const int32_t* row_perm,
                                                                int N, int mode) {
-    // mode 0: no row order; 1: reorder through shared memory; 2: scattered
-    // stores (a row of y larger than shared memory)
+    // mode 0: no row order; 1: reorder through shared memory (N floats)
     extern __shared__ __align__(16) float srow[];
     pdl_launch_dependents();
     pdl_wait();   // the partial sums come from the kernel before
@@ -541,7 +538,7 @@ __global__ void __launch_bounds__(FINISH_THREADS) k_finish_rows(float* y, const 
             float v = pr[i];
             for (int sp = 1; sp < splits; ++sp) v += pr[(size_t)sp * split_stride + i];
             if (mode == 0) yr[i] = v;
-            else (mode == 1 ? srow : yr)[row_perm[i]] = v;
+            else srow[row_perm[i]] = v;
         }
     }
     if (mode != 1) return;

@@ -180,9 +180,12 @@ bool perm_ok(const int32_t* p, int n) {
 
 inline mpq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MPQ_OK : MPQ_ERR_CUDA; }
 
+constexpr size_t kUnpermMaxBytes = 200 * 1024;   // one row of y in shared memory
+
 // Tensor-core launch shape: 256-token tiles beyond one 128-token tile, and
 // the k blocks split across CTAs (partial sums reduced by k_finish_rows)
-// while the grid stays within one wave of 148 SMs.
+// while the grid stays within one wave of 148 SMs.  A split grid has at most
+// 74 tiles of 128 rows, so a row of y then always fits in shared memory.
 struct PrefillShape {
     int BN, tiles_n, tiles_m, splits, kb_per_split;
 };
@@ -194,7 +197,9 @@ PrefillShape prefill_shape(int N, int K, int M) {
     ps.tiles_m = (M + ps.BN - 1) / ps.BN;
     const int ctas = ps.tiles_n * ps.tiles_m;
     int splits = 1;
-    while (splits < 8 && ctas * splits * 2 <= 148 && KB / (splits * 2) >= 4) splits *= 2;
+    while (splits < 8 && ctas * splits * 2 <= 148 && KB / (splits * 2) >= 4 &&
+           (size_t)N * 4 <= kUnpermMaxBytes)
+        splits *= 2;
     ps.kb_per_split = (KB + splits - 1) / splits;
     ps.splits = (KB + ps.kb_per_split - 1) / ps.kb_per_split;
     return ps;
@@ -261,7 +266,6 @@ std::atomic<uint64_t> g_decode_attr8{0};
 std::atomic<uint64_t> g_prefill_attr{0};
 std::atomic<uint64_t> g_prefill_attr256{0};
 std::atomic<uint64_t> g_unperm_attr{0};
-constexpr size_t kUnpermMaxBytes = 200 * 1024;   // one row of y in shared memory
 
 // cuTensorMapEncodeTiled from the driver, looked up through the runtime.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -496,8 +500,8 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
             cudaLaunchConfig_t uc{};
             uc.gridDim = dim3((unsigned)M);
             uc.blockDim = dim3(FINISH_THREADS);
-            // 0: no row order, 1: reorder through shared memory, 2: scattered stores
-            const int mode = !layer->row_perm ? 0 : row_fits ? 1 : 2;
+            // 0: no row order, 1: reorder through shared memory
+            const int mode = layer->row_perm ? 1 : 0;
             uc.dynamicSmemBytes = mode == 1 ? (size_t)layer->N * 4 : 0;
             uc.stream = s;
             uc.attrs = pdl;

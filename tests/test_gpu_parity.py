@@ -215,9 +215,9 @@ def test_linear_host_entry_point(mpq, oracle):
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("cfg,proj,Ms", [(3, 0, (1, 8, 16, 32)), (3, 2, (1, 8)),
                                          (4, 1, (1, 4, 16)), (4, 3, (1,)),
-                                         # tensor-core path at the prefill sizes: 128-token
-                                         # tiles (512, ragged 700) and 256-token tiles
-                                         # (2048, ragged 1100)
+                                         # tensor-core path at the prefill sizes, 256-token
+                                         # tiles: k split in 2 (q at 512), in 4 (k at ragged
+                                         # 700), not split (2048, down at ragged 1100)
                                          (5, 0, (512, 2048)), (5, 1, (700,)), (5, 6, (1100,))])
 def test_full_size_sampled(mpq, oracle, cfg, proj, Ms):
     L = synth.config_layer(cfg, proj)
@@ -232,3 +232,36 @@ def test_full_size_sampled(mpq, oracle, cfg, proj, Ms):
         y = run_linear(mpq, P, x)
         y_ref, bnd = oracle.linear_rows(R, x, rows)
         assert_y_close(y[:, rows], y_ref, bnd)
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core launch shapes (M > 16): split-K with a ragged last split, with
+# and without the row reordering, one 128- or 256-token tile, an odd number
+# of block rows, and a layer too wide for the reordering kernel's
+# shared-memory row (the epilogue then scatters through row_perm itself).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K,M,perm,sampled", [
+    (512, 128 * 11, 40, True, False),      # 2 splits of 6 + 5 k blocks
+    (256, 128 * 37, 129, True, False),     # 8 splits of 5 (last 2), 256-token tile, ragged
+    (384, 1024, 64, False, False),         # 2 splits, no row order
+    (384, 512, 48, False, False),          # no split, no row order: direct stores
+    (320, 512, 17, True, False),           # smallest tensor-core batch, odd number of row blocks
+    (51264, 256, 20, True, True),          # a row of y beyond shared memory
+    (2048, 128 * 24, 300, True, False),    # 256-token tiles, 2 rows of them (ragged), 4 splits
+])
+def test_tensor_core_shapes(mpq, oracle, N, K, M, perm, sampled):
+    L = synth.make_layer("tc", N, K, 3.0, 4000 + N + K + M, "random")
+    if not perm:
+        L.row_perm = None
+        L.col_perm = None
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    x = synth.make_x(4100 + M, M, K)
+    y = run_linear(mpq, P, x)
+    if sampled:
+        rows = np.sort(np.random.default_rng(N).choice(N, 128, replace=False)).astype(np.int32)
+        y_ref, bnd = oracle.linear_rows(R, x, rows)
+        assert_y_close(y[:, rows], y_ref, bnd)
+    else:
+        y_ref, bnd = oracle.linear(R, x)
+        assert_y_close(y, y_ref, bnd)
