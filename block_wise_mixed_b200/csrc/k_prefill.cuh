@@ -44,28 +44,32 @@ constexpr int PF_DQ_WARPS = 16;                  // warps 2 .. 17
 constexpr int PF_WARPS = PF_DQ_WARPS + 3;
 constexpr int PF_THREADS = PF_WARPS * 32;
 constexpr int PF_BM = 128;       // weight rows per tile (2 block rows)
-constexpr int PF_A_STAGES = 2;   // dequantized weight tiles
 constexpr int PF_A_BYTES = PF_BM * 256;           // 128 rows x 128 fp16
 constexpr int PF_C_BYTES = 2 * 8192 + 4 * 128;    // two payloads + 2 x (scales, zeros)
 
 // Tokens per tile: 128, or 256 for large batches (each dequantized weight
 // tile then feeds twice the tensor-core work).  Activation stages hold half
 // a k block (64 columns) so that both fit in shared memory.
+//
+// With 256 tokens a k block's MMAs take about as long as its dequantization,
+// so three weight stages keep the dequantizing warps one k block further
+// ahead (two code stages make the room).
 template <int BN>
 struct PfCfg {
+    static constexpr int A_STAGES = BN == 256 ? 3 : 2;   // dequantized weight tiles
     static constexpr int B_STAGES = BN == 256 ? 3 : 4;   // half-k-block activation stages (from L2)
     static constexpr int B_BYTES = BN * 128;              // BN tokens x 64 fp16
-    static constexpr int C_STAGES = BN == 256 ? 3 : 5;   // packed codes (from HBM)
+    static constexpr int C_STAGES = BN == 256 ? 2 : 5;   // packed codes (from HBM)
     static constexpr uint32_t TMEM_COLS = BN;             // fp32 accumulator columns
 };
 
 template <int BN>
 struct PrefillSmem {
-    uint8_t a[PF_A_STAGES][PF_A_BYTES];    // 1024-aligned (offset 0)
+    uint8_t a[PfCfg<BN>::A_STAGES][PF_A_BYTES];    // 1024-aligned (offset 0)
     uint8_t b[PfCfg<BN>::B_STAGES][PfCfg<BN>::B_BYTES];
     uint8_t c[PfCfg<BN>::C_STAGES][PF_C_BYTES];
-    uint64_t full_a[PF_A_STAGES];
-    uint64_t empty_a[PF_A_STAGES];
+    uint64_t full_a[PfCfg<BN>::A_STAGES];
+    uint64_t empty_a[PfCfg<BN>::A_STAGES];
     uint64_t full_b[PfCfg<BN>::B_STAGES];
     uint64_t empty_b[PfCfg<BN>::B_STAGES];
     uint64_t full_c[PfCfg<BN>::C_STAGES];
@@ -73,7 +77,7 @@ struct PrefillSmem {
     uint64_t d_full;
     uint32_t tmem_base;
     volatile int abort_flag;
-    // per tile: code_off, sz_off, bits of the two block rows, KB entries each
+    // followed by the widths of the tile's blocks: [2][KB] bytes
 };
 
 struct PrefillParams {
@@ -166,8 +170,11 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int kc) {
 // Dequantizes groups [g0, g0+4) (8 codes each) of row rr of one block of
 // width B into the A tile row r: w_hat = (q - z) * s in fp16.  A warp covers
 // 8 whole rows (lane = row * 4 + quarter), so the lanes' code bytes are one
-// contiguous run of shared memory (one conflict-free vector load each), and
-// their 16-byte A chunks fall four to a bank group.
+// contiguous run of shared memory (one conflict-free vector load each).  The
+// quarters 2 and 3 take their groups in the order 2, 3, 0, 1: chunks kc and
+// kc + 8 of a row share a bank group under the 128B swizzle, and with this
+// order the 8 lanes of each store phase (two rows x four quarters) hit 8
+// different bank groups.
 template <int P>
 __device__ __forceinline__ void load_part(const uint8_t* p, uint32_t (&w)[P]) {
     if (P == 1) {
@@ -205,8 +212,29 @@ __device__ __forceinline__ void dequant_row_part(const uint8_t* payload, const _
         const uint2 v = *reinterpret_cast<const uint2*>(payload + 64 * 16 * P0 + rr * 32 + 2 * g0);
         e[0] = v.x; e[P1 > 1 ? 1 : 0] = v.y;
     }
+    // group order: step gi takes group gi ^ sw (sw = 2 for quarters 2, 3)
+    const int sw = (g0 & 8) ? 2 : 0;
+    if (P0 == 4 || P0 == 8) {
+        constexpr int H = P0 / 2;   // words of two groups
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            const uint32_t lo = d[i], hi = d[i + H];
+            d[i] = sw ? hi : lo;
+            d[i + H] = sw ? lo : hi;
+        }
+    } else if (P0 == 2) {
+        const uint32_t lo = d[0], hi = d[P0 > 1 ? 1 : 0];
+        d[0] = sw ? hi : lo;
+        d[P0 > 1 ? 1 : 0] = sw ? lo : hi;
+    }
+    if (P1 == 2) {
+        const uint32_t lo = e[0], hi = e[P1 > 1 ? 1 : 0];
+        e[0] = sw ? hi : lo;
+        e[P1 > 1 ? 1 : 0] = sw ? lo : hi;
+    }
 #pragma unroll
     for (int gi = 0; gi < 4; ++gi) {
+        const int g = gi ^ sw;   // the group this step takes
         uint32_t o[4];
         if (P0 == 4) {
             ext4(d[gi], k[0], k[1], o);
@@ -215,11 +243,11 @@ __device__ __forceinline__ void dequant_row_part(const uint8_t* payload, const _
         } else if (P0 == 2) {
             ext2(d[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, k, o);
         } else {
-            ext1(d[0], gi | (4 << 4) | (gi << 8) | (4 << 12), k, o);
+            ext1(d[0], g | (4 << 4) | (g << 8) | (4 << 12), k, o);
         }
         if (P1 > 0) {
             uint32_t h[4];
-            if (P1 == 1) ext1_hi<P0>(e[0], gi | (4 << 4) | (gi << 8) | (4 << 12), h);
+            if (P1 == 1) ext1_hi<P0>(e[0], g | (4 << 4) | (g << 8) | (4 << 12), h);
             else ext2_hi(e[gi >> 1], (gi & 1) ? 0x4342 : 0x4140, h);
 #pragma unroll
             for (int j = 0; j < 4; ++j) o[j] = h2_bits(__hadd2(bits_h2(o[j]), bits_h2(h[j])));
@@ -229,7 +257,7 @@ __device__ __forceinline__ void dequant_row_part(const uint8_t* payload, const _
         w.y = h2_bits(__hmul2(bits_h2(o[1]), s2));
         w.z = h2_bits(__hmul2(bits_h2(o[2]), s2));
         w.w = h2_bits(__hmul2(bits_h2(o[3]), s2));
-        *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + gi)) = w;
+        *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + g)) = w;
     }
 }
 
@@ -237,6 +265,7 @@ template <int BN>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     using Cfg = PfCfg<BN>;
+    constexpr int PF_A_STAGES = Cfg::A_STAGES;
     constexpr int PF_C_STAGES = Cfg::C_STAGES;
     constexpr int PF_B_STAGES = Cfg::B_STAGES;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -247,7 +276,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     // arithmetic on smem_raw keeps the shared address space for the compiler
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     PrefillSmem<BN>& S = *reinterpret_cast<PrefillSmem<BN>*>(base);
-    uint32_t* tab = reinterpret_cast<uint32_t*>(base + sizeof(PrefillSmem<BN>));  // [2][KB][3]
+    uint8_t* tbits = base + sizeof(PrefillSmem<BN>);   // [2][KB] block widths
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tiles = p.tiles_n * p.tiles_m;
@@ -260,16 +289,11 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     const int kb0 = split * p.kb_per_split;
     const int KB = max(0, min(p.KB, kb0 + p.kb_per_split) - kb0);
 
-    // stage this tile's table entries: tab[(h*KB + kb)*3 + {0,1,2}]
+    // stage the widths of this CTA's blocks: tbits[h*KB + kb]
     for (int i = tid; i < 2 * KB; i += PF_THREADS) {
         const int h = i / KB, kb = i % KB;
         const int nb = nb0 + h;
-        uint32_t co = 0, so = 0, bits = 0;
-        if (nb < p.NB) {
-            const mpq_block e = p.table[(size_t)nb * p.KB + kb0 + kb];
-            co = e.code_off; so = e.sz_off; bits = e.bits;
-        }
-        tab[3 * i] = co; tab[3 * i + 1] = so; tab[3 * i + 2] = bits;
+        tbits[i] = nb < p.NB ? (uint8_t)p.table[(size_t)nb * p.KB + kb0 + kb].bits : (uint8_t)0;
     }
     if (tid == 0) {
         for (int s = 0; s < PF_A_STAGES; ++s) {
@@ -304,34 +328,57 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
         set_error(p.err, MPQ_ERR_TIMEOUT);
         S.abort_flag = 1;
     };
-    auto bits_of = [&](int h, int kb) -> uint32_t { return tab[3 * (h * KB + kb) + 2]; };
+    auto bits_of = [&](int h, int kb) -> uint32_t { return tbits[h * KB + kb]; };
 
     if (warp == 0) {
         // -------------------- producer of the packed codes --------------------
         // runs as far ahead as the code stages allow (the weights do not
-        // depend on the prologue kernel)
-        if (lane == 0) {
-            int a = 0;
-            for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
+        // depend on the prologue kernel); the code and scale offsets of 32 k
+        // blocks are read from the table at a time, one k block per lane
+        int a = 0;
+        bool stop = false;
+        for (int kbb = 0; kbb < KB && !stop; kbb += 32) {
+            uint32_t co0 = 0, so0 = 0, co1 = 0, so1 = 0;
+            if (kbb + lane < KB) {
+                const size_t e = (size_t)nb0 * p.KB + kb0 + kbb + lane;
+                co0 = p.table[e].code_off; so0 = p.table[e].sz_off;
+                if (nb0 + 1 < p.NB) { co1 = p.table[e + p.KB].code_off; so1 = p.table[e + p.KB].sz_off; }
+            }
+            const int n = min(32, KB - kbb);
+            for (int j = 0; j < n; ++j) {
+                const int kb = kbb + j;
                 const uint32_t b0 = bits_of(0, kb), b1 = bits_of(1, kb);
                 if ((b0 | b1) == 0) continue;
-                const int sc = a % PF_C_STAGES;
-                const uint32_t pc = (uint32_t)(a / PF_C_STAGES) & 1u;
-                if (!mbar_wait_bounded(&S.empty_c[sc], pc ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
-                uint32_t bytes = (b0 ? 1024u * b0 + 256u : 0u) + (b1 ? 1024u * b1 + 256u : 0u);
-                mbar_arrive_expect_tx(&S.full_c[sc], bytes);
-                uint8_t* cst = S.c[sc];
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t b = h ? b1 : b0;
-                    if (!b) continue;
-                    const uint32_t co = tab[3 * (h * KB + kb)], so = tab[3 * (h * KB + kb) + 1];
-                    bulk_g2s(cst + h * 8192, p.codes + co, 1024u * b, &S.full_c[sc]);
-                    bulk_g2s(cst + 16384 + h * 256, p.scales + so, 128u, &S.full_c[sc]);
-                    bulk_g2s(cst + 16384 + h * 256 + 128, p.zeros + so, 128u, &S.full_c[sc]);
+                const uint32_t c0 = __shfl_sync(0xffffffffu, co0, j), s0 = __shfl_sync(0xffffffffu, so0, j);
+                const uint32_t c1 = __shfl_sync(0xffffffffu, co1, j), s1 = __shfl_sync(0xffffffffu, so1, j);
+                bool ok = true;
+                if (lane == 0) {
+                    const int sc = a % PF_C_STAGES;
+                    const uint32_t pc = (uint32_t)(a / PF_C_STAGES) & 1u;
+                    ok = !S.abort_flag && mbar_wait_bounded(&S.empty_c[sc], pc ^ 1u, DEC_WAIT_NS);
+                    if (ok) {
+                        const uint32_t bytes = (b0 ? 1024u * b0 + 256u : 0u) + (b1 ? 1024u * b1 + 256u : 0u);
+                        mbar_arrive_expect_tx(&S.full_c[sc], bytes);
+                        uint8_t* cst = S.c[sc];
+                        if (b0) {
+                            bulk_g2s(cst, p.codes + c0, 1024u * b0, &S.full_c[sc]);
+                            bulk_g2s(cst + 16384, p.scales + s0, 128u, &S.full_c[sc]);
+                            bulk_g2s(cst + 16384 + 128, p.zeros + s0, 128u, &S.full_c[sc]);
+                        }
+                        if (b1) {
+                            bulk_g2s(cst + 8192, p.codes + c1, 1024u * b1, &S.full_c[sc]);
+                            bulk_g2s(cst + 16384 + 256, p.scales + s1, 128u, &S.full_c[sc]);
+                            bulk_g2s(cst + 16384 + 384, p.zeros + s1, 128u, &S.full_c[sc]);
+                        }
+                    } else if (!S.abort_flag) {
+                        timed_out();
+                    }
                 }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
                 ++a;
             }
         }
+        __syncwarp();
     } else if (warp == PF_WARPS - 1) {
         // ------------------- producer of the activation tiles -----------------
         pdl_wait();   // x' comes from the prologue kernel

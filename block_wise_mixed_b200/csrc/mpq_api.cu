@@ -193,6 +193,8 @@ PrefillShape prefill_shape(int N, int K, int M) {
     PrefillShape ps{};
     const int NB = N / 64, KB = K / 128;
     ps.BN = M > 128 ? 256 : 128;
+    // 256-token stages leave shared memory for the widths of up to ~440 k blocks
+    if (ps.BN == 256 && sizeof(PrefillSmem<256>) + 1024 + (size_t)2 * KB > (size_t)227 * 1024) ps.BN = 128;
     ps.tiles_n = (NB + 1) / 2;
     ps.tiles_m = (M + ps.BN - 1) / ps.BN;
     const int ctas = ps.tiles_n * ps.tiles_m;
@@ -296,7 +298,7 @@ bool make_tmap_fp16(CUtensorMap* map, const void* ptr, int K, int rows, int box_
 
 template <int BN>
 size_t prefill_smem_bytes(int KB) {
-    return sizeof(PrefillSmem<BN>) + 1024 + (size_t)2 * KB * 12;
+    return sizeof(PrefillSmem<BN>) + 1024 + (size_t)2 * KB;
 }
 
 
