@@ -74,6 +74,8 @@ def lib():
         L.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
         L.mpq_pack_workspace_size.restype = sz
         L.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
+        L.mpq_pack_timed.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P,
+                                     P, P]
         L.mpq_linear_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
         L.mpq_linear_workspace_size.restype = sz
         L.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
@@ -86,7 +88,7 @@ def lib():
         L.mpq_check.argtypes = [P, P]
         L.mpq_status_string.argtypes = [ctypes.c_int]
         L.mpq_status_string.restype = ctypes.c_char_p
-        for f in ("mpq_plan", "mpq_pack", "mpq_linear", "mpq_linear_timed", "mpq_linear_host",
+        for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_timed", "mpq_linear_host",
                   "mpq_check"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -173,8 +175,10 @@ def alloc_layer(L: Layout, device, has_row_perm: bool, has_col_perm: bool) -> Pa
 
 
 def pack(W, bits: np.ndarray, row_perm=None, col_perm=None, ws=None, check=True,
-         stream=None) -> PackedLayer:
-    """mpq_pack.  W: torch bf16 (or int16/uint16 bit patterns) N x K on cuda."""
+         stream=None, ev_begin=None, ev_end=None) -> PackedLayer:
+    """mpq_pack (mpq_pack_timed when torch.cuda.Event objects are given: they
+    bracket the quantize kernel alone).  W: torch bf16 (or int16/uint16 bit
+    patterns) N x K on cuda."""
     import torch
     N, K = W.shape
     bits = np.ascontiguousarray(bits, dtype=np.uint8).reshape(-1)
@@ -186,8 +190,13 @@ def pack(W, bits: np.ndarray, row_perm=None, col_perm=None, ws=None, check=True,
         ws = torch.empty(lib().mpq_pack_workspace_size(ctypes.byref(L)), dtype=torch.uint8,
                          device=W.device)
     Wc = W.contiguous()
-    st = lib().mpq_pack(ctypes.byref(L), Wc.data_ptr(), _np_ptr(bits), _np_ptr(rp), _np_ptr(cp),
-                        ctypes.byref(P.c), ws.data_ptr(), ws.numel(), _stream(stream))
+    if ev_begin is None and ev_end is None:
+        st = lib().mpq_pack(ctypes.byref(L), Wc.data_ptr(), _np_ptr(bits), _np_ptr(rp), _np_ptr(cp),
+                            ctypes.byref(P.c), ws.data_ptr(), ws.numel(), _stream(stream))
+    else:
+        st = lib().mpq_pack_timed(ctypes.byref(L), Wc.data_ptr(), _np_ptr(bits), _np_ptr(rp),
+                                  _np_ptr(cp), ctypes.byref(P.c), ws.data_ptr(), ws.numel(),
+                                  _stream(stream), _event(ev_begin), _event(ev_end))
     _raise(st, "mpq_pack")
     if check:
         _raise(lib().mpq_check(ws.data_ptr(), _stream(stream)), "mpq_pack (device)")
@@ -211,6 +220,15 @@ def linear(layer: PackedLayer, x, out=None, ws=None, stream=None):
                           ws.data_ptr(), ws.numel(), _stream(stream))
     _raise(st, "mpq_linear")
     return out
+
+
+def _event(ev):
+    """The cudaEvent_t handle of a torch.cuda.Event (or None)."""
+    if ev is None:
+        return None
+    if ev.cuda_event == 0:   # torch creates the CUDA event on first record
+        ev.record()
+    return ctypes.c_void_p(ev.cuda_event)
 
 
 def linear_timed(layer: PackedLayer, x, out, ws, ev_begin, ev_end, stream=None):

@@ -26,7 +26,7 @@ constexpr int kMaxUnits = 148 * DEC_CTAS_PER_SM * DEC_WARPS;   // one run per re
 constexpr uint64_t kMinUnitCost = 4096; // cost units (bytes) per run, at least
 constexpr int kMaxDecodeTokens = DEC_MAX_TOKENS;   // tokens per decode launch
 constexpr int kDecodeMaxM = 16;         // larger batches take the tensor-core kernel
-constexpr int kPackRowsPerCta = 16;
+constexpr int kPackRowsPerCta = 1;
 
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -327,6 +327,14 @@ size_t mpq_pack_workspace_size(const mpq_layout*) { return 256; }
 mpq_status mpq_pack(const mpq_layout* L, const void* W_dev, const uint8_t* bits_host,
                     const int32_t* row_perm_host, const int32_t* col_perm_host,
                     const mpq_layer* out, void* ws, size_t ws_bytes, void* stream) {
+    return mpq_pack_timed(L, W_dev, bits_host, row_perm_host, col_perm_host, out, ws, ws_bytes,
+                          stream, nullptr, nullptr);
+}
+
+mpq_status mpq_pack_timed(const mpq_layout* L, const void* W_dev, const uint8_t* bits_host,
+                          const int32_t* row_perm_host, const int32_t* col_perm_host,
+                          const mpq_layer* out, void* ws, size_t ws_bytes, void* stream,
+                          void* ev_begin, void* ev_end) {
     if (!L || !W_dev || !bits_host || !out) return MPQ_ERR_ARG;
     mpq_layout chk;
     std::vector<mpq_block> table;
@@ -363,7 +371,13 @@ mpq_status mpq_pack(const mpq_layout* L, const void* W_dev, const uint8_t* bits_
                             (size_t)L->K * 4, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, 4, s);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
-    if (L->bit_total == 0) return MPQ_OK;   // nothing to quantize
+    if (ev_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s) != cudaSuccess)
+        return MPQ_ERR_CUDA;
+    if (L->bit_total == 0) {   // nothing to quantize
+        if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
+            return MPQ_ERR_CUDA;
+        return MPQ_OK;
+    }
 
     PackParams p{};
     p.W = static_cast<const uint16_t*>(W_dev);
@@ -384,7 +398,9 @@ mpq_status mpq_pack(const mpq_layout* L, const void* W_dev, const uint8_t* bits_
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
     const int grid = (L->N + kPackRowsPerCta - 1) / kPackRowsPerCta;
     k_pack<<<grid, PACK_THREADS, smem, s>>>(p);
-    return cuda_status(cudaGetLastError());
+    e = cudaGetLastError();
+    if (e == cudaSuccess && ev_end) e = cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s);
+    return cuda_status(e);
 }
 
 size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M) {

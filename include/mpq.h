@@ -159,6 +159,17 @@ mpq_status mpq_pack(const mpq_layout* L, const void* W_dev,
                     const int32_t* col_perm_host, const mpq_layer* out,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* mpq_pack with two optional cudaEvent_t handles (NULL = none): ev_begin is
+ * recorded on `stream` after the host planning and the table / schedule /
+ * permutation uploads, right before the quantize kernel, and ev_end right
+ * after it, so a caller can time the kernel alone.  Same arguments, results
+ * and errors as mpq_pack. */
+mpq_status mpq_pack_timed(const mpq_layout* L, const void* W_dev,
+                          const uint8_t* bits_host, const int32_t* row_perm_host,
+                          const int32_t* col_perm_host, const mpq_layer* out,
+                          void* ws, size_t ws_bytes, void* stream, void* ev_begin,
+                          void* ev_end);
+
 /* Workspace bytes that mpq_linear needs for M tokens. */
 size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
 
