@@ -151,9 +151,12 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle as it stands
 # ---------------------------------------------------------------------------
-def oracle_baseline(layer, x, min_seconds=10.0, rows=None):
+def oracle_baseline(layer, x, min_seconds=10.0, rows=None, threads=None):
+    """The oracle's linear timed on the host: all cores (threads=None) or a
+    given number of OpenMP threads."""
     from oracle import oracle
     R = oracle.pack(layer.W, layer.bits, layer.row_perm, layer.col_perm)
+    prev = oracle.set_threads(threads) if threads else None
     if rows is None:
         rows = np.arange(layer.N, dtype=np.int32)
     n = 0
@@ -164,12 +167,14 @@ def oracle_baseline(layer, x, min_seconds=10.0, rows=None):
         el = time.perf_counter() - t0
         if el >= min_seconds:
             break
+    if prev is not None:
+        oracle.set_threads(prev)
     frac = len(rows) / layer.N
     T = (layer.N // 64) * (layer.K // 128)
     nbytes = algorithmic_bytes(layer.N, layer.K, x.shape[0], R.codes.size * frac,
                                R.scales.size * frac, T * frac, layer.row_perm is not None,
                                layer.col_perm is not None)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cores = threads or int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": nbytes * n / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": "%d calls of the fp64 oracle's linear on %d of %d output rows "
                       "(dequant + dot), %.1f s" % (n, len(rows), layer.N, el),
@@ -291,11 +296,27 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     torch.cuda.synchronize(device)
     e2e_ms = reduce_max_over_ranks(h0.elapsed_time(h1), world, device) / steps
 
+    # one cold call: L2 flushed by writing a buffer twice its size, then a
+    # single mpq_linear between events (launch latency included)
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    cold = []
+    for i in range(3):
+        flush.fill_(i + 1)
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        mpq.linear(reps[i % R], x, y, ws)
+        c1.record(stream)
+        torch.cuda.synchronize(device)
+        cold.append(c0.elapsed_time(c1))
+    del flush
+    cold_ms = float(np.median(cold))
+
     kbytes = (lay.codes_bytes + 4 * lay.n_sz + 16 * T + 4 * (L.N if L.row_perm is not None else 0)
               + 2 * M * L.K + 4 * M * L.N)
     out = dict(N=L.N, K=L.K, M=M, avg_bits=float(L.bits.mean()), f0=float((L.bits == 0).mean()),
                replicas=R, l2_bytes=int(l2), bytes=nbytes, kernel_bytes=kbytes,
-               ms_step=ms_step, kernel_ms=k_ms, e2e_ms=e2e_ms, clocks=clocks,
+               ms_step=ms_step, kernel_ms=k_ms, e2e_ms=e2e_ms, cold_ms=cold_ms, clocks=clocks,
                launches_per_step=1 + (M + 7) // 8, n_units=lay.n_units,
                h2d=M * L.K * 2, d2h=M * L.N * 4)
     del reps
@@ -370,10 +391,16 @@ def run_gpu(args):
                 "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"]},
         "clocks": r["clocks"],
         "gpu_launches": args.steps * r["launches_per_step"],
+        # one call after an L2 flush, launch latency included (not the headline)
+        "cold": {"us": round(r["cold_ms"] * 1e3, 2),
+                 "GBps": round(r["bytes"] / (r["cold_ms"] * 1e-3) / 1e9, 1)},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         xb = synth.make_x(synth.seed_of(99, 0), M, layer.K)
         res["cpu_baseline"] = oracle_baseline(layer, xb, min_seconds=args.cpu_seconds)
+        one = oracle_baseline(layer, xb, min_seconds=args.cpu_seconds, threads=1)
+        res["cpu_baseline"]["single_thread"] = {"value": one["value"], "cores": 1,
+                                                "sample": one["sample"]}
     if args.extra and rank == 0:
         res["extra"] = run_extra(mpq, args, device, peaks)
         res["extra"]["tensor_core_llama3_8b_layer"] = run_tensor_core(mpq, args, device, peaks)
@@ -524,6 +551,8 @@ def run_reference(args):
     for _ in range(args.steps):
         oracle.linear_rows(R, x, rows)
     el = time.perf_counter() - t0
+    if prev is not None:
+        oracle.set_threads(prev)
     frac = len(rows) / layer.N
     T = (layer.N // 64) * (layer.K // 128)
     nbytes = algorithmic_bytes(layer.N, layer.K, M, R.codes.size * frac, R.scales.size * frac,

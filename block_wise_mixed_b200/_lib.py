@@ -80,6 +80,9 @@ def lib():
         L.mpq_linear_workspace_size.restype = sz
         L.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
         L.mpq_linear_timed.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P, P, P]
+        L.mpq_linear_typed_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_int]
+        L.mpq_linear_typed_workspace_size.restype = sz
+        L.mpq_linear_typed.argtypes = [ctypes.POINTER(Layer), P, i32, P, ctypes.c_int, P, sz, P]
         L.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
         L.mpq_linear_host_workspace_size.restype = sz
         L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
@@ -88,7 +91,7 @@ def lib():
         L.mpq_check.argtypes = [P, P]
         L.mpq_status_string.argtypes = [ctypes.c_int]
         L.mpq_status_string.restype = ctypes.c_char_p
-        for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_timed", "mpq_linear_host",
+        for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_typed", "mpq_linear_timed", "mpq_linear_host",
                   "mpq_check"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -207,17 +210,30 @@ def linear_workspace_size(layer: PackedLayer, M: int) -> int:
     return lib().mpq_linear_workspace_size(ctypes.byref(layer.c), M)
 
 
-def linear(layer: PackedLayer, x, out=None, ws=None, stream=None):
-    """mpq_linear: y (fp32, M x N) = x (bf16, M x K, cuda) * dequant(W)^T."""
+Y_F32, Y_BF16 = 0, 1   # mpq_ydtype
+
+
+def linear_typed_workspace_size(layer: PackedLayer, M: int, ydtype: int = Y_F32) -> int:
+    return lib().mpq_linear_typed_workspace_size(ctypes.byref(layer.c), M, ydtype)
+
+
+def linear(layer: PackedLayer, x, out=None, ws=None, stream=None, ydtype: int = Y_F32):
+    """mpq_linear: y (M x N) = x (bf16, M x K, cuda) * dequant(W)^T; y fp32, or
+    bf16 (mpq_linear_typed, MPQ_Y_BF16) with ydtype=Y_BF16."""
     import torch
     M, K = x.shape
     if out is None:
-        out = torch.empty((M, layer.N), dtype=torch.float32, device=x.device)
+        dt = torch.bfloat16 if ydtype == Y_BF16 else torch.float32
+        out = torch.empty((M, layer.N), dtype=dt, device=x.device)
     if ws is None:
-        ws = torch.empty(max(linear_workspace_size(layer, M), 256), dtype=torch.uint8,
+        ws = torch.empty(max(linear_typed_workspace_size(layer, M, ydtype), 256), dtype=torch.uint8,
                          device=x.device)
-    st = lib().mpq_linear(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(),
-                          ws.data_ptr(), ws.numel(), _stream(stream))
+    if ydtype == Y_F32:
+        st = lib().mpq_linear(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(),
+                              ws.data_ptr(), ws.numel(), _stream(stream))
+    else:
+        st = lib().mpq_linear_typed(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(), ydtype,
+                                    ws.data_ptr(), ws.numel(), _stream(stream))
     _raise(st, "mpq_linear")
     return out
 

@@ -17,6 +17,7 @@
 #include "k_pack.cuh"
 #include "k_prefill.cuh"
 #include "k_xprep.cuh"
+#include "k_ycast.cuh"
 
 using namespace mpq;
 
@@ -411,6 +412,43 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M) {
 mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
                       void* ws, size_t ws_bytes, void* stream) {
     return mpq_linear_timed(layer, x_dev, M, y_dev, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+size_t mpq_linear_typed_workspace_size(const mpq_layer* layer, int32_t M, mpq_ydtype ydt) {
+    if (!layer || M < 0) return 0;
+    const size_t base = round256(carve_linear(nullptr, layer, M).bytes);
+    // bf16: the fp32 product is kept in the workspace before rounding
+    return ydt == MPQ_Y_BF16 ? base + (size_t)M * layer->N * 4 : base;
+}
+
+mpq_status mpq_linear_typed(const mpq_layer* layer, const void* x_dev, int32_t M, void* y_dev,
+                            mpq_ydtype ydt, void* ws, size_t ws_bytes, void* stream) {
+    if (ydt == MPQ_Y_F32)
+        return mpq_linear(layer, x_dev, M, static_cast<float*>(y_dev), ws, ws_bytes, stream);
+    if (ydt != MPQ_Y_BF16) return MPQ_ERR_ARG;
+    mpq_status st = check_layer(layer);
+    if (st != MPQ_OK) return st;
+    if (M < 0) return MPQ_ERR_SHAPE;
+    if (M == 0) return MPQ_OK;
+    if (!x_dev || !y_dev) return MPQ_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
+    const size_t base = round256(carve_linear(nullptr, layer, M).bytes);
+    const size_t n = (size_t)M * layer->N;
+    if (ws_bytes < base + n * 4) return MPQ_ERR_WORKSPACE;
+    float* y32 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + base);
+    st = mpq_linear(layer, x_dev, M, y32, ws, base, stream);
+    if (st != MPQ_OK) return st;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c{};
+    c.gridDim = dim3((unsigned)std::min<size_t>((n / 4 + YCAST_THREADS - 1) / YCAST_THREADS + 1, 148 * 8));
+    c.blockDim = dim3(YCAST_THREADS);
+    c.stream = static_cast<cudaStream_t>(stream);
+    c.attrs = pdl;
+    c.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&c, k_y_to_bf16, (const float*)y32,
+                                          static_cast<uint16_t*>(y_dev), n));
 }
 
 mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,

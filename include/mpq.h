@@ -88,6 +88,12 @@ typedef enum {
     MPQ_ERR_TIMEOUT = 9     /* a bounded device wait ran out (device)       */
 } mpq_status;
 
+/* Element type of y for mpq_linear_typed. */
+typedef enum {
+    MPQ_Y_F32 = 0,          /* fp32: the graded output (mpq_linear)          */
+    MPQ_Y_BF16 = 1          /* bf16, round-to-nearest-even of the fp32 y     */
+} mpq_ydtype;
+
 /* One block of the table (16 bytes). */
 typedef struct {
     uint32_t code_off;    /* byte offset of the payload in `codes` (0 if 0-bit) */
@@ -188,6 +194,18 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
  * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT. */
 mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M,
                       float* y_dev, void* ws, size_t ws_bytes, void* stream);
+
+/* mpq_linear with a choice of output type.  MPQ_Y_F32 is mpq_linear itself
+ * (y_dev is float*).  MPQ_Y_BF16 writes y_dev as bf16 bit patterns (uint16,
+ * M x N row-major): the fp32 result of mpq_linear, kept in the workspace,
+ * rounded to nearest-even.  This is a convenience for callers that feed a bf16
+ * model: the rounding alone (up to 2^-9 relative) exceeds the fp32 path's
+ * error bars.  ws must hold mpq_linear_typed_workspace_size(layer, M, ydt)
+ * bytes.  Errors: those of mpq_linear; ARG for an unknown ydt. */
+size_t mpq_linear_typed_workspace_size(const mpq_layer* layer, int32_t M, mpq_ydtype ydt);
+mpq_status mpq_linear_typed(const mpq_layer* layer, const void* x_dev, int32_t M,
+                            void* y_dev, mpq_ydtype ydt, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /* mpq_linear that also records two CUDA events (cudaEvent_t as void*; either
  * may be NULL) on `stream`: ev_begin right before the first launch of the

@@ -40,11 +40,18 @@
  * rounding mode).  Compile without -ffast-math.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
 #include "mpq_oracle.h"
+
+int mpqo_set_threads(int n) {
+    const int prev = omp_get_max_threads();
+    omp_set_num_threads(n < 1 ? 1 : n);
+    return prev;
+}
 
 /* ------------------------------------------------------------------------ */
 /* Number formats                                                            */

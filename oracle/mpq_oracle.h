@@ -35,6 +35,10 @@ typedef struct {
     const int32_t *row_perm, *col_perm;   /* NULL = identity */
 } mpqo_packed;
 
+/* Threads of the OpenMP loops (n >= 1); returns the previous count.  Only
+ * the timing of the oracle uses it; results do not depend on it. */
+int mpqo_set_threads(int n);
+
 double mpqo_bf16_to_f64(uint16_t b);
 double mpqo_f16_to_f64(uint16_t h);
 int mpqo_bits_valid(int b);

@@ -66,6 +66,7 @@ def lib():
         _lib = ctypes.CDLL(build())
         P = ctypes.c_void_p
         i32 = ctypes.c_int32
+        _lib.mpqo_set_threads.argtypes = [ctypes.c_int]
         _lib.mpqo_plan.argtypes = [i32, i32, P, ctypes.POINTER(_Layout), P]
         _lib.mpqo_quantize_group.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P]
         _lib.mpqo_pack.argtypes = [i32, i32, P, P, P, P, P, P, P, P]
@@ -196,6 +197,11 @@ def linear_dense(x_bf16: np.ndarray, What: np.ndarray):
 def linear(P: Packed, x_bf16: np.ndarray):
     """The layer's output for x (bf16 bits, M x K): (y, bound), float64 M x N."""
     return linear_dense(x_bf16, dequant(P))
+
+
+def set_threads(n: int) -> int:
+    """OpenMP threads of the oracle's loops (for timing); returns the previous count."""
+    return lib().mpqo_set_threads(int(n))
 
 
 def linear_rows(P: Packed, x_bf16: np.ndarray, rows: np.ndarray):

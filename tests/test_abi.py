@@ -109,3 +109,24 @@ def test_linear_host_validation(lib):
     assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), None, 4, P(16), P(256), need, None)] == "MPQ_ERR_ARG"
     bad = B.Layer(100, 256, L.n_units, 0, 16, 16, 16, 16, 16, None, None)
     assert B.STATUS[lib.mpq_linear(ctypes.byref(bad), P(16), 4, P(16), P(256), need, None)] == "MPQ_ERR_SHAPE"
+
+
+def test_linear_typed_host_validation(lib):
+    """mpq_linear_typed: the bf16 workspace holds the fp32 product on top of
+    mpq_linear's; host-side checks return before any launch."""
+    L = B.plan(128, 256, np.array([1, 2, 3, 4], np.uint8))
+    layer = _fake_layer(L)
+    P = ctypes.c_void_p
+    M = 4
+    f32 = lib.mpq_linear_typed_workspace_size(ctypes.byref(layer), M, B.Y_F32)
+    b16 = lib.mpq_linear_typed_workspace_size(ctypes.byref(layer), M, B.Y_BF16)
+    plain = lib.mpq_linear_workspace_size(ctypes.byref(layer), M)
+    assert f32 >= plain and f32 % 256 == 0 and f32 - plain < 256
+    assert b16 == f32 + M * L.N * 4
+    typed = lib.mpq_linear_typed
+    assert B.STATUS[typed(ctypes.byref(layer), P(16), M, P(16), 2, P(256), b16, None)] == "MPQ_ERR_ARG"
+    assert B.STATUS[typed(ctypes.byref(layer), P(16), M, P(16), B.Y_BF16, P(256), b16 - 1,
+                          None)] == "MPQ_ERR_WORKSPACE"
+    assert B.STATUS[typed(ctypes.byref(layer), P(16), M, None, B.Y_BF16, P(256), b16,
+                          None)] == "MPQ_ERR_ARG"
+    assert typed(ctypes.byref(layer), P(16), 0, P(16), B.Y_BF16, P(256), b16, None) == 0

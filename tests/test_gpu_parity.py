@@ -265,3 +265,33 @@ def test_tensor_core_shapes(mpq, oracle, N, K, M, perm, sampled):
     else:
         y_ref, bnd = oracle.linear(R, x)
         assert_y_close(y, y_ref, bnd)
+
+
+# ---------------------------------------------------------------------------
+# bf16 output (mpq_linear_typed, MPQ_Y_BF16): exactly the round-to-nearest-
+# even of the fp32 product, on the decode and the tensor-core paths.
+# ---------------------------------------------------------------------------
+def bf16_rne_bits(y32: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even of fp32 values to bf16 bit patterns (finite input)."""
+    u = np.ascontiguousarray(y32, np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return r.astype(np.uint16)
+
+
+@pytest.mark.parametrize("N,K,M", [(256, 512, 3), (384, 1024, 64), (4096, 4096, 1)])
+def test_linear_bf16_output(mpq, oracle, N, K, M):
+    import torch
+    L = synth.make_layer("y16", N, K, 2.5, 5000 + N + M, "random")
+    P = pack_gpu(mpq, L)
+    x = synth.make_x(5100 + M, M, K)
+    y32 = run_linear(mpq, P, x)
+    y16 = mpq.linear(P, dev(x), ydtype=mpq.Y_BF16)
+    torch.cuda.synchronize()
+    assert y16.dtype == torch.bfloat16 and tuple(y16.shape) == (M, N)
+    got = y16.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, bf16_rne_bits(y32))
+    # against the oracle: its bound plus the bf16 rounding of the value
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    y_ref, bnd = oracle.linear(R, x)
+    yb = synth.bf16_bits_to_f32(got).astype(np.float64)
+    assert np.all(np.abs(yb - y_ref) <= PER_OUT * bnd + 2.0 ** -8 * np.abs(y_ref) + 1e-30)
