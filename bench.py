@@ -203,6 +203,19 @@ def build_replicas(mpq, P, R):
     return reps
 
 
+def launches_per_call(lay, M, has_row_perm):
+    """Kernels one mpq_linear call launches (the library's dispatch rule):
+    M <= 16 -- the activation prologue unless M == 1 on a layer whose runs
+    hold at most two blocks on average (the decode kernel then builds its own
+    activation records), plus one decode launch per 8 tokens; M > 16 -- the
+    prologue, the tensor-core kernel and, when the rows are reordered, the
+    reordering kernel (split-K partials too)."""
+    if M <= 16:
+        fused = M == 1 and lay.NB * lay.KB <= 2 * lay.n_units
+        return (0 if fused else 1) + (M + 7) // 8
+    return 2 + (1 if has_row_perm else 0)
+
+
 def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sampler=None,
                quick=False):
     """Times `steps` mpq_linear calls over L2-busting replicas of one layer.
@@ -222,7 +235,7 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     x_bits = synth.make_x(synth.seed_of(99, 0), M, L.K)
     x = torch.from_numpy(x_bits.view(np.int16)).to(device)
     y = torch.empty((M, L.N), dtype=torch.float32, device=device)
-    ws = torch.empty(mpq.linear_workspace_size(P, M), dtype=torch.uint8, device=device)
+    ws = torch.zeros(mpq.linear_workspace_size(P, M), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     for i in range(max(warmup, 3)):
         mpq.linear(reps[i % R], x, y, ws)
@@ -283,7 +296,7 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     # end to end through the host entry point (pinned host x and y)
     xh = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
     yh = torch.empty((M, L.N), dtype=torch.float32).pin_memory()
-    wsh = torch.empty(mpq.linear_host_workspace_size(P, M), dtype=torch.uint8, device=device)
+    wsh = torch.zeros(mpq.linear_host_workspace_size(P, M), dtype=torch.uint8, device=device)
     for i in range(3):
         mpq.linear_host(reps[i % R], xh, yh, wsh)
     torch.cuda.synchronize(device)
@@ -317,7 +330,7 @@ def time_layer(mpq, layer_spec, M, steps, warmup, world, device, soak_s=1.0, sam
     out = dict(N=L.N, K=L.K, M=M, avg_bits=float(L.bits.mean()), f0=float((L.bits == 0).mean()),
                replicas=R, l2_bytes=int(l2), bytes=nbytes, kernel_bytes=kbytes,
                ms_step=ms_step, kernel_ms=k_ms, e2e_ms=e2e_ms, cold_ms=cold_ms, clocks=clocks,
-               launches_per_step=1 + (M + 7) // 8, n_units=lay.n_units,
+               launches_per_step=launches_per_call(lay, M, L.row_perm is not None), n_units=lay.n_units,
                h2d=M * L.K * 2, d2h=M * L.N * 4)
     del reps
     torch.cuda.empty_cache()
@@ -428,7 +441,7 @@ def time_prefill(mpq, L, M, steps, device):
     reps = build_replicas(mpq, P, R)
     x = torch.from_numpy(synth.make_x(synth.seed_of(98, 0), M, L.K).view(np.int16)).to(device)
     y = torch.empty((M, L.N), dtype=torch.float32, device=device)
-    ws = torch.empty(mpq.linear_workspace_size(P, M), dtype=torch.uint8, device=device)
+    ws = torch.zeros(mpq.linear_workspace_size(P, M), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     for i in range(3):
         mpq.linear(reps[i % R], x, y, ws)

@@ -226,7 +226,7 @@ def linear(layer: PackedLayer, x, out=None, ws=None, stream=None, ydtype: int = 
         dt = torch.bfloat16 if ydtype == Y_BF16 else torch.float32
         out = torch.empty((M, layer.N), dtype=dt, device=x.device)
     if ws is None:
-        ws = torch.empty(max(linear_typed_workspace_size(layer, M, ydtype), 256), dtype=torch.uint8,
+        ws = torch.zeros(max(linear_typed_workspace_size(layer, M, ydtype), 256), dtype=torch.uint8,
                          device=x.device)
     if ydtype == Y_F32:
         st = lib().mpq_linear(ctypes.byref(layer.c), x.data_ptr(), M, out.data_ptr(),

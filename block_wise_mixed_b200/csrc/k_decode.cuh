@@ -64,6 +64,8 @@ struct DecodeParams {
     const uint16_t* zeros;
     const int32_t* row_perm;
     const uint8_t* xq;        // k_xprep_decode records: [KB][XQD_REC * M_total]
+    const uint16_t* x;        // bf16 x [M_total][K] (the fused one-token path reads it)
+    const int32_t* col_perm;  // [K] or null (fused path)
     float* y;                 // [M_total][N]
     float* partial;           // [slots][Mg][64]
     uint32_t* counters;       // [NB] arrivals per block row
@@ -85,6 +87,7 @@ constexpr int DEC_MAX_TOKENS = 8;
 struct DecWarp {
     uint8_t ring[DEC_RING];
     int32_t rows[64];         // output index of each row of the current block row
+    __half xw[128];           // fused path: the block's x' slice, column order
     uint64_t full[DEC_SLOTS];
     uint4 zero16[4];          // zero B fragments for lanes beyond the token count
 };
@@ -348,10 +351,67 @@ __device__ __noinline__ void finish_shared_row(const float* __restrict__ slots, 
 }
 
 // ---------------------------------------------------------------------------
+// Fused activation record (one token, no prologue kernel): the record that
+// k_xprep_decode would write for block column kb and piece-width variant vv,
+// built by the warp into `rec` (shared memory, XQD_VAR bytes): the slice
+// x[m][col_perm[128kb + c]], c = 0..127, scaled by its power of two 2^e and
+// converted to fp16, paired in the variant's column order, then
+// F = 2^(24 - e) -- the same arithmetic as k_xprep_decode.  cp holds the
+// column indices 128kb + 4 lane .. +3 (after col_perm).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int4 fused_cols(const DecodeParams& p, uint32_t kb, int lane) {
+    const int c0 = (int)kb * 128 + 4 * lane;
+    if (!p.col_perm) return make_int4(c0, c0 + 1, c0 + 2, c0 + 3);
+    return __ldg(reinterpret_cast<const int4*>(p.col_perm + c0));
+}
+
+__device__ __forceinline__ void fused_record(const DecodeParams& p, int4 cp, int vv, uint8_t* rec,
+                                             __half* xw, int lane) {
+    const uint16_t* xr = p.x + (size_t)p.m0 * p.K;
+    float v[4];
+    v[0] = __uint_as_float((uint32_t)xr[cp.x] << 16);
+    v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
+    v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
+    v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
+    float amax = 0.f;
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+        const float a = fabsf(v[e4]);
+        amax = (a > amax || a != a) ? a : amax;   // NaN-propagating max
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, amax, off);
+        amax = (o > amax || o != o) ? o : amax;
+    }
+    int e = 0;
+    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -103), 126);
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) xw[4 * lane + e4] = __float2half_rn(ldexpf(v[e4], e));
+    __syncwarp();
+    // lane -> quad lane tq = lane / 8, pairs 2 (lane % 8), +1
+    const int tq = lane >> 3, pi0 = 2 * (lane & 7);
+    uint32_t o[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        int ca, cb;
+        xqd_pair_cols(vv, pi0 + i, ca, cb);
+        o[i] = h2_bits(__halves2half2(xw[32 * tq + ca], xw[32 * tq + cb]));
+    }
+    *reinterpret_cast<uint2*>(rec + tq * 64 + pi0 * 4) = make_uint2(o[0], o[1]);
+    if (lane == 0) *reinterpret_cast<float*>(rec + 256) = ldexpf(1.f, 24 - e);
+    // generic writes into the ring, later overwritten by bulk copies
+    fence_proxy_async_smem();
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // The kernel.  ONE_TOKEN: the launch has Mg == 1 (only C-fragment column 0
 // carries data, so the per-block epilogue handles half the elements).
+// FUSED_X (with ONE_TOKEN): no prologue kernel; each block's activation
+// record is built by the warp from x (fused_record).
 // ---------------------------------------------------------------------------
-template <bool ONE_TOKEN>
+template <bool ONE_TOKEN, bool FUSED_X = false>
 // At most 112 registers: four CTAs then leave room in the register file for
 // the next launch's activation-prologue CTAs to become resident early.
 __global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
@@ -473,12 +533,13 @@ __global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
             if (lane == 0) {
                 fence_proxy_async_smem();
                 uint64_t* bar = &W.full[slot];
-                mbar_arrive_expect_tx(bar, size);
+                // the fused path builds the activation record itself
+                mbar_arrive_expect_tx(bar, FUSED_X ? size - x_bytes : size);
                 uint8_t* dst = W.ring + off;
                 bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
                 bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
                 bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
-                if (xq_ready) bulk_g2s(dst + 1024u * b + 256u, p.xq + xo, x_bytes, bar);
+                if (!FUSED_X && xq_ready) bulk_g2s(dst + 1024u * b + 256u, p.xq + xo, x_bytes, bar);
             }
             if (lane == (int)slot) { qe_t = tt; qe_bits = b; qe_off = off; qe_end = start + size; qe_x = xo; }
             r_head = start + size;
@@ -491,14 +552,24 @@ __global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
     // Weights do not depend on the prologue kernel: start streaming them, then
     // wait for x' (programmatic dependent launch) and add its copies.
     issue_more();
+    // fused path: the column order of the first block's slice is static, so
+    // it is read before waiting for the kernel that writes x
+    int4 cp_pref = make_int4(0, 0, 0, 0);
+    uint32_t cp_kb = 0xFFFFFFFFu;
+    if (FUSED_X && q_head != q_tail) {
+        cp_kb = __shfl_sync(0xffffffffu, qe_t, q_head % DEC_SLOTS) % KB;
+        cp_pref = fused_cols(p, cp_kb, lane);
+    }
     pdl_wait();
     xq_ready = true;
-    for (uint32_t k = q_head; k < q_tail; ++k) {
-        const uint32_t slot = k % DEC_SLOTS;
-        const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
-        const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
-        const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
-        if (lane == 0) bulk_g2s(W.ring + ko + 1024u * kbits + 256u, p.xq + kx, x_bytes, &W.full[slot]);
+    if (!FUSED_X) {
+        for (uint32_t k = q_head; k < q_tail; ++k) {
+            const uint32_t slot = k % DEC_SLOTS;
+            const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
+            const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
+            const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
+            if (lane == 0) bulk_g2s(W.ring + ko + 1024u * kbits + 256u, p.xq + kx, x_bytes, &W.full[slot]);
+        }
     }
 
     const uint32_t nb_first = t0 / KB, nb_last = (t1 - 1) / KB;
@@ -536,6 +607,12 @@ __global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
             if (!aborted) {
                 const uint8_t* stage = W.ring + foff;
                 const uint8_t* xs = stage + 1024u * fb + 256u;
+                if (FUSED_X) {
+                    const uint32_t kb = ft % KB;
+                    const int4 cp = (kb == cp_kb) ? cp_pref : fused_cols(p, kb, lane);
+                    fused_record(p, cp, variant_of(lo_width((int)fb)), W.ring + foff + 1024u * fb + 256u,
+                                 W.xw, lane);
+                }
                 // this lane's B fragments: token g, quad lane t; zeros beyond Mg
                 uint32_t bf[16];
                 load_bfrag((uint32_t)g < Mg ? xs + g * XQD_VAR + t * 64

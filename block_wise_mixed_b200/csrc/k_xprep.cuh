@@ -17,7 +17,7 @@
 //   XP_PREFILL: [M][K] half, K contiguous, each 128-column group permuted so
 //               that position 2*(4i+j)+h holds column 8i+j+4h -- the order in
 //               which the tensor-core kernel's dequantization emits weights.
-// Block 0 also clears the workspace error word.
+// Block 0 also clears the decode kernel's per-block-row counters (when given).
 //
 // k_xprep_decode (below) is the small-batch variant; its layout is described
 // there.
@@ -35,7 +35,6 @@ struct XprepParams {
     float* tok_scale;          // [M] = 2^-e_m
     uint32_t* counters;        // [n_counters] cleared by block 0 (may be null)
     int n_counters;
-    uint32_t* err;             // cleared by block 0 (may be null)
     int M, K;
 };
 
@@ -50,7 +49,6 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
     __shared__ float red[XPREP_THREADS / 32];
     const int m = blockIdx.x, tid = threadIdx.x, K = p.K;
     if (m == 0) {
-        if (tid == 0 && p.err) *p.err = 0u;
         if (p.counters)
             for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
     }
@@ -140,8 +138,7 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
 // variant v = 0..3 (p = 1, 2, 4, 8) and token m, XQD_VAR = 272 bytes:
 //   [t = 0..3][pi = 0..15] half2 (256 B), then F as float4 (F, 0, 0, 0)
 // so one variant of a token group is one contiguous run of 272*Mg bytes.
-// Block 0 also clears the workspace error word and the decode kernel's
-// per-block-row counters.
+// Block 0 also clears the decode kernel's per-block-row counters.
 // ---------------------------------------------------------------------------
 constexpr int XQD_VAR = 272;                 // one variant of one token: fragments + F
 constexpr int XQD_REC = 4 * XQD_VAR;
@@ -175,7 +172,6 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
     if (p.col_perm && active) cp = *reinterpret_cast<const int4*>(p.col_perm + c0);
     pdl_wait();   // the kernel before may still read the workspace or write x
     if (blockIdx.x == 0) {
-        if (tid == 0 && p.err) *p.err = 0u;
         if (p.counters)
             for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
     }

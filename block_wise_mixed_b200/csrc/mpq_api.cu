@@ -266,6 +266,7 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
 }
 std::atomic<uint64_t> g_decode_attr{0};
 std::atomic<uint64_t> g_decode_attr8{0};
+std::atomic<uint64_t> g_decode_attr_f{0};
 std::atomic<uint64_t> g_prefill_attr{0};
 std::atomic<uint64_t> g_prefill_attr256{0};
 std::atomic<uint64_t> g_unperm_attr{0};
@@ -467,6 +468,10 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
 
     const bool use_tc = M > kDecodeMaxM;
     if (!use_tc && (uint64_t)KB * (uint64_t)M * XQD_REC >= (1ull << 32)) return MPQ_ERR_SHAPE;
+    // one token on a layer whose runs hold at most two blocks on average: the
+    // decode kernel builds its activation records itself (no prologue kernel,
+    // one launch boundary less on this latency-bound path)
+    const bool fused = !use_tc && M == 1 && (size_t)NB * KB <= 2 * (size_t)layer->n_units;
     XprepParams xp{};
     xp.x = static_cast<const uint16_t*>(x_dev);
     xp.col_perm = layer->col_perm;
@@ -474,7 +479,6 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     xp.tok_scale = w.tok_scale;
     xp.counters = w.counters;
     xp.n_counters = NB;
-    xp.err = w.err;
     xp.M = M;
     xp.K = layer->K;
     // Every launch may overlap the end of the kernel before it (programmatic
@@ -493,10 +497,12 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
         xp.counters = nullptr;
         xc.gridDim = dim3((unsigned)M);
         e = cudaLaunchKernelEx(&xc, k_xprep<XP_PREFILL>, xp);
-    } else {
+    } else if (!fused) {
         const int items = KB * M, per = XPREP_THREADS / 32;
         xc.gridDim = dim3((unsigned)((items + per - 1) / per));
         e = cudaLaunchKernelEx(&xc, k_xprep_decode, xp);
+    } else {
+        e = cudaSuccess;
     }
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
 
@@ -573,6 +579,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
 
     e = ensure_smem_attr(k_decode<true>, (int)sizeof(DecSmem), g_decode_attr);
     if (e == cudaSuccess) e = ensure_smem_attr(k_decode<false>, (int)sizeof(DecSmem), g_decode_attr8);
+    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<true, true>, (int)sizeof(DecSmem), g_decode_attr_f);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
     DecodeParams dp{};
     dp.codes = static_cast<const uint8_t*>(layer->codes);
@@ -582,6 +589,8 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     dp.zeros = layer->zeros;
     dp.row_perm = layer->row_perm;
     dp.xq = reinterpret_cast<const uint8_t*>(w.xq);
+    dp.x = static_cast<const uint16_t*>(x_dev);
+    dp.col_perm = layer->col_perm;
     dp.y = y_dev;
     dp.partial = w.partial;
     dp.counters = w.counters;
@@ -608,8 +617,9 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     for (int m0 = 0; m0 < M; m0 += kMaxDecodeTokens) {
         dp.m0 = m0;
         dp.Mg = std::min(kMaxDecodeTokens, M - m0);
-        e = dp.Mg == 1 ? cudaLaunchKernelEx(&cfg, k_decode<true>, dp)
-                       : cudaLaunchKernelEx(&cfg, k_decode<false>, dp);
+        e = fused ? cudaLaunchKernelEx(&cfg, k_decode<true, true>, dp)
+            : dp.Mg == 1 ? cudaLaunchKernelEx(&cfg, k_decode<true>, dp)
+                         : cudaLaunchKernelEx(&cfg, k_decode<false>, dp);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
     }
     if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
@@ -650,6 +660,8 @@ mpq_status mpq_check(const void* ws, void* stream) {
     uint32_t err = 0;
     if (cudaStreamSynchronize(s) != cudaSuccess) return MPQ_ERR_CUDA;
     if (cudaMemcpy(&err, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MPQ_ERR_CUDA;
+    // reported: clear it for the calls that follow
+    if (err != 0u && cudaMemset(const_cast<void*>(ws), 0, 4) != cudaSuccess) return MPQ_ERR_CUDA;
     return static_cast<mpq_status>(err);
 }
 

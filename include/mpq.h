@@ -60,7 +60,9 @@
  *   - Errors that the host can see are returned at once and nothing is
  *     launched.  Errors found in device data (non-finite W, a group with no
  *     representable scale) or a device wait that ran out are written to an
- *     error word at the start of the workspace; mpq_check() reports them.
+ *     error word at the start of the workspace: the first such error since
+ *     the workspace was zero-filled or since the last mpq_check(), which
+ *     reports and clears it (mpq_pack clears it when it starts).
  *   - A launch failure returns MPQ_ERR_CUDA.
  *   - Limits: N % 64 == 0, K % 128 == 0, N, K > 0, K <= 65536 when a column
  *     permutation is given, codes_bytes < 2^32; M >= 0 (M == 0 is a no-op).
@@ -186,7 +188,10 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
  *   x_dev   bf16 bit patterns, M x K row-major (device).
  *   y_dev   fp32, M x N row-major, original output order (device).
  *   ws      device workspace of >= mpq_linear_workspace_size(layer, M) bytes,
- *           256-byte aligned; its contents need no initialization.
+ *           256-byte aligned, zero-filled before its first use (e.g.
+ *           cudaMemset); every call that ends without a device error leaves
+ *           the parts that must start at zero at zero, so it can be reused
+ *           as is (zero it again after a device error).
  * Uses a memory-bound decode kernel for M <= 16 and a tensor-core kernel for
  * larger M.  Non-finite x gives non-finite y (no error).  Activations are
  * moved into fp16 by exact powers of two; for M <= 16 that needs
@@ -220,7 +225,8 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
  * M x K) into the workspace, runs mpq_linear and copies y back to y_host
  * (fp32, M x N), all on `stream`; returns after enqueueing (synchronize the
  * stream before reading y_host).  Use pinned host memory for asynchrony.
- * ws must hold mpq_linear_host_workspace_size(layer, M) bytes. */
+ * ws must hold mpq_linear_host_workspace_size(layer, M) bytes and follows
+ * the same zero-fill rule as mpq_linear's. */
 size_t mpq_linear_host_workspace_size(const mpq_layer* layer, int32_t M);
 mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host,
                            int32_t M, float* y_host, void* ws,
@@ -240,8 +246,8 @@ mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host,
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
- *   All calls share the one array, which keeps the last call's contents
- *   (the parts that must start at zero are cleared by each call): calls
+ *   All calls share the one array, which starts zeroed and keeps the last
+ *   call's contents (the parts that must start at zero are left at zero): calls
  *   that overlap on the GPU -- on different streams, or from different
  *   threads -- race and give wrong results.  Serialize them.
  *   Device-side errors go to the array's error word, which mpq_check cannot
@@ -250,8 +256,10 @@ mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host,
 mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t M,
                               float* y_dev, void* stream);
 
-/* Synchronizes `stream` and returns the device error word stored in `ws` by
- * the last mpq_pack / mpq_linear on that workspace (MPQ_OK if none). */
+/* Synchronizes `stream` and returns the device error word of `ws`: the first
+ * device error of the mpq_linear calls on that workspace since it was
+ * zero-filled or since the previous mpq_check, or of the last mpq_pack
+ * (MPQ_OK if none); then clears it. */
 mpq_status mpq_check(const void* ws, void* stream);
 
 /* Human-readable name of a status. */

@@ -202,7 +202,7 @@ def test_linear_host_entry_point(mpq, oracle):
     x = synth.make_x(synth.seed_of(1, 0), 3, L.K)
     xh = torch.from_numpy(x.view(np.int16)).pin_memory()
     yh = torch.empty((3, L.N), dtype=torch.float32).pin_memory()
-    ws = torch.empty(mpq.linear_host_workspace_size(P, 3), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(mpq.linear_host_workspace_size(P, 3), dtype=torch.uint8, device="cuda")
     mpq.linear_host(P, xh, yh, ws)
     torch.cuda.synchronize()
     y_ref, bnd = oracle.linear(R, x)
@@ -295,3 +295,25 @@ def test_linear_bf16_output(mpq, oracle, N, K, M):
     y_ref, bnd = oracle.linear(R, x)
     yb = synth.bf16_bits_to_f32(got).astype(np.float64)
     assert np.all(np.abs(yb - y_ref) <= PER_OUT * bnd + 2.0 ** -8 * np.abs(y_ref) + 1e-30)
+
+
+def test_workspace_reuse(mpq):
+    """One zero-filled workspace serves a mix of calls (one-token layers whose
+    decode builds its own activation records, the prologue-kernel path, the
+    tensor-core path): each result equals the same call on a fresh workspace,
+    so every call leaves the workspace's counters at zero; no device error."""
+    import torch
+    from block_wise_mixed_b200 import _lib
+    small = synth.config_layer(2, 0)                       # one block per run: fused
+    big = synth.config_layer(3, 0)                         # ~3 blocks per run: prologue kernel
+    Ps, Pb = pack_gpu(mpq, small), pack_gpu(mpq, big)
+    calls = [(Ps, 1), (Pb, 1), (Ps, 3), (Ps, 1), (Pb, 40), (Ps, 1), (Pb, 2), (Ps, 1)]
+    size = max(mpq.linear_workspace_size(P, M) for P, M in calls)
+    ws = torch.zeros(size, dtype=torch.uint8, device="cuda")
+    for i, (P, M) in enumerate(calls):
+        x = dev(synth.make_x(600 + i, M, P.K))
+        got = mpq.linear(P, x, ws=ws)
+        want = mpq.linear(P, x)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), i
+    assert _lib.lib().mpq_check(ws.data_ptr(), None) == 0
