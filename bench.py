@@ -417,6 +417,9 @@ def run_gpu(args):
     if args.extra and rank == 0:
         res["extra"] = run_extra(mpq, args, device, peaks)
         res["extra"]["tensor_core_llama3_8b_layer"] = run_tensor_core(mpq, args, device, peaks)
+        # q, k, v of Llama-2-7B (three seeded 4096x4096 layers) in one call
+        qkv = [synth.config_layer(2, 0, replica=r) for r in range(3)]
+        res["extra"]["group_llama2_7b_qkv_M1"] = time_group(mpq, qkv, min(args.steps, 200), device)
         res["extra"]["pack_llama3_8b_layer"] = run_pack(mpq, device, peaks)
     if world > 1:
         import torch.distributed as dist
@@ -525,6 +528,60 @@ def run_pack(mpq, device, peaks):
     gbs = tot_bytes / (tot_us * 1e-6) / 1e9
     return {"layer_gpu_us": round(tot_us, 1), "GBps": round(gbs, 1),
             "frac": round(gbs / peaks["hbm_gbs"], 4), "projections": per}
+
+
+def time_group(mpq, specs, steps, device):
+    """Layers that share x at M=1: mpq_linear_group (one launch when every
+    layer's decode builds its own activation records) against one mpq_linear
+    per layer, each as a CUDA graph over L2-busting replicas."""
+    import torch
+    from block_wise_mixed_b200 import synth
+    Ps = []
+    for L in specs:
+        W = torch.from_numpy(L.W.view(np.int16)).to(device)
+        Ps.append(mpq.pack(W, L.bits, L.row_perm, L.col_perm))
+        del W
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    per = sum(P.layout.codes_bytes + 4 * P.layout.n_sz for P in Ps)
+    R = int(max(2, min(256, np.ceil(4 * l2 / max(per, 1)))))
+    reps = [build_replicas(mpq, P, R) for P in Ps]
+    x = torch.from_numpy(synth.make_x(synth.seed_of(97, 0), 1, specs[0].K).view(np.int16)).to(device)
+    ys = [torch.empty((1, L.N), dtype=torch.float32, device=device) for L in specs]
+    wsg = torch.zeros(mpq.linear_group_workspace_size(Ps, 1), dtype=torch.uint8, device=device)
+    wss = torch.zeros(max(mpq.linear_workspace_size(P, 1) for P in Ps), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def run(grouped, r):
+        layers = [rp[r % R] for rp in reps]
+        if grouped:
+            mpq.linear_group(layers, x, ys, wsg)
+        else:
+            for P, y in zip(layers, ys):
+                mpq.linear(P, x, y, wss)
+
+    out = {}
+    for grouped in (True, False):
+        for r in range(5):
+            run(grouped, r)
+        torch.cuda.synchronize(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for r in range(steps):
+                run(grouped, r)
+        graph.replay()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream); graph.replay(); e1.record(stream)
+        torch.cuda.synchronize(device)
+        out["grouped_us" if grouped else "separate_us"] = round(e0.elapsed_time(e1) * 1e3 / steps, 2)
+        del graph
+    nbytes = sum(algorithmic_bytes(L.N, L.K, 1, P.layout.codes_bytes, P.layout.n_sz,
+                                   P.layout.NB * P.layout.KB, L.row_perm is not None,
+                                   L.col_perm is not None) for L, P in zip(specs, Ps))
+    out["GBps_grouped"] = round(nbytes / (out["grouped_us"] * 1e-6) / 1e9, 1)
+    del reps
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_extra(mpq, args, device, peaks):

@@ -83,6 +83,9 @@ def lib():
         L.mpq_linear_typed_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_int]
         L.mpq_linear_typed_workspace_size.restype = sz
         L.mpq_linear_typed.argtypes = [ctypes.POINTER(Layer), P, i32, P, ctypes.c_int, P, sz, P]
+        L.mpq_linear_group_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, i32]
+        L.mpq_linear_group_workspace_size.restype = sz
+        L.mpq_linear_group.argtypes = [ctypes.POINTER(Layer), i32, P, i32, P, P, sz, P]
         L.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
         L.mpq_linear_host_workspace_size.restype = sz
         L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
@@ -91,7 +94,8 @@ def lib():
         L.mpq_check.argtypes = [P, P]
         L.mpq_status_string.argtypes = [ctypes.c_int]
         L.mpq_status_string.restype = ctypes.c_char_p
-        for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_typed", "mpq_linear_timed", "mpq_linear_host",
+        for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_typed",
+                  "mpq_linear_group", "mpq_linear_timed", "mpq_linear_host",
                   "mpq_check"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -236,6 +240,39 @@ def linear(layer: PackedLayer, x, out=None, ws=None, stream=None, ydtype: int = 
                                     ws.data_ptr(), ws.numel(), _stream(stream))
     _raise(st, "mpq_linear")
     return out
+
+
+GROUP_MAX = 8   # MPQ_GROUP_MAX
+
+
+def _layer_array(layers):
+    arr = (Layer * len(layers))()
+    for i, P in enumerate(layers):
+        arr[i] = P.c
+    return arr
+
+
+def linear_group_workspace_size(layers, M: int) -> int:
+    return lib().mpq_linear_group_workspace_size(_layer_array(layers), len(layers), M)
+
+
+def linear_group(layers, x, outs=None, ws=None, stream=None):
+    """mpq_linear_group: y_i (fp32, M x N_i) = x (bf16, M x K, cuda) * dequant(W_i)^T
+    for layers that share K; one launch for the group when M == 1 on short-run
+    layers.  Returns the list of outputs."""
+    import torch
+    M, K = x.shape
+    if outs is None:
+        outs = [torch.empty((M, P.N), dtype=torch.float32, device=x.device) for P in layers]
+    arr = _layer_array(layers)
+    if ws is None:
+        ws = torch.zeros(max(lib().mpq_linear_group_workspace_size(arr, len(layers), M), 256),
+                         dtype=torch.uint8, device=x.device)
+    ptrs = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
+    st = lib().mpq_linear_group(arr, len(layers), x.data_ptr(), M, ptrs, ws.data_ptr(), ws.numel(),
+                                _stream(stream))
+    _raise(st, "mpq_linear_group")
+    return outs
 
 
 def _event(ev):

@@ -406,33 +406,13 @@ __device__ __forceinline__ void fused_record(const DecodeParams& p, int4 cp, int
 }
 
 // ---------------------------------------------------------------------------
-// The kernel.  ONE_TOKEN: the launch has Mg == 1 (only C-fragment column 0
-// carries data, so the per-block epilogue handles half the elements).
-// FUSED_X (with ONE_TOKEN): no prologue kernel; each block's activation
-// record is built by the warp from x (fused_record).
+// One warp's run u of the layer p (the body of the decode kernels below).
 // ---------------------------------------------------------------------------
-template <bool ONE_TOKEN, bool FUSED_X = false>
-// At most 112 registers: four CTAs then leave room in the register file for
-// the next launch's activation-prologue CTAs to become resident early.
-__global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+template <bool ONE_TOKEN, bool FUSED_X>
+__device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, int u, int lane) {
     const int g = lane >> 2, t = lane & 3;
-    DecWarp& W = S.w[warp];
-    const int u = blockIdx.x * DEC_WARPS + warp;
     const uint32_t KB = (uint32_t)p.KB;
     const uint32_t lt_mask = (1u << lane) - 1u;
-
-    // the next kernel in the stream may launch now: it waits (griddepcontrol)
-    // for this grid before it touches memory this kernel uses
-    pdl_launch_dependents();
-    if (lane == 0) {
-        for (int s = 0; s < DEC_SLOTS; ++s) mbar_init(&W.full[s], 1);
-        fence_mbar_init();
-    }
-    if (lane < 4) W.zero16[lane] = make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();
     if (u >= p.n_units) return;
 
     // ---- the unit descriptor: lane i holds word i ----
@@ -689,6 +669,59 @@ __global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
                           p.N, W.rows, lane);
         if (lane == 0) p.counters[nb] = 0u;   // ready for the next launch
     }
+}
+
+
+// ---------------------------------------------------------------------------
+// The kernels.  ONE_TOKEN: the launch has Mg == 1 (only C-fragment column 0
+// carries data, so the per-block epilogue handles half the elements).
+// FUSED_X (with ONE_TOKEN): no prologue kernel; each block's activation
+// record is built by the warp from x (fused_record).  Every warp works
+// alone (no CTA-wide barrier): warp u of the grid takes run u.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ DecWarp& decode_prologue(uint8_t* smem_raw, int warp, int lane) {
+    DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
+    DecWarp& W = S.w[warp];
+    // the next kernel in the stream may launch now: it waits (griddepcontrol)
+    // for this grid before it touches memory this kernel uses
+    pdl_launch_dependents();
+    if (lane == 0) {
+        for (int s = 0; s < DEC_SLOTS; ++s) mbar_init(&W.full[s], 1);
+        fence_mbar_init();
+    }
+    if (lane < 4) W.zero16[lane] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+    return W;
+}
+
+template <bool ONE_TOKEN, bool FUSED_X = false>
+// At most 112 registers: four CTAs then leave room in the register file for
+// the next launch's activation-prologue CTAs to become resident early.
+__global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    DecWarp& W = decode_prologue(smem_raw, warp, lane);
+    decode_warp<ONE_TOKEN, FUSED_X>(p, W, (int)blockIdx.x * DEC_WARPS + warp, lane);
+}
+
+// Several layers that share x in one launch (one token, fused activation
+// records): the runs of layer l are warps unit_begin[l] .. unit_begin[l+1]-1.
+constexpr int DEC_GROUP_MAX = 8;
+struct DecodeGroup {
+    DecodeParams layer[DEC_GROUP_MAX];
+    int unit_begin[DEC_GROUP_MAX + 1];
+    int n;
+};
+
+__global__ void __maxnreg__(DEC_MAX_REGS) k_decode_group(const __grid_constant__ DecodeGroup gp) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    DecWarp& W = decode_prologue(smem_raw, warp, lane);
+    const int v = (int)blockIdx.x * DEC_WARPS + warp;
+    if (v >= gp.unit_begin[gp.n]) return;
+    int l = 0;
+    while (l + 1 < gp.n && v >= gp.unit_begin[l + 1]) ++l;
+    decode_warp<true, true>(gp.layer[l], W, v - gp.unit_begin[l], lane);
 }
 
 }  // namespace mpq

@@ -267,6 +267,7 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
 std::atomic<uint64_t> g_decode_attr{0};
 std::atomic<uint64_t> g_decode_attr8{0};
 std::atomic<uint64_t> g_decode_attr_f{0};
+std::atomic<uint64_t> g_decode_attr_g{0};
 std::atomic<uint64_t> g_prefill_attr{0};
 std::atomic<uint64_t> g_prefill_attr256{0};
 std::atomic<uint64_t> g_unperm_attr{0};
@@ -452,26 +453,53 @@ mpq_status mpq_linear_typed(const mpq_layer* layer, const void* x_dev, int32_t M
                                           static_cast<uint16_t*>(y_dev), n));
 }
 
-mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
-                            void* ws, size_t ws_bytes, void* stream, void* ev_begin,
-                            void* ev_end) {
-    mpq_status st = check_layer(layer);
-    if (st != MPQ_OK) return st;
-    if (M < 0) return MPQ_ERR_SHAPE;
-    if (M == 0) return MPQ_OK;
-    if (!x_dev || !y_dev) return MPQ_ERR_ARG;
-    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
-    LinearWs w = carve_linear(ws, layer, M);
-    if (ws_bytes < w.bytes) return MPQ_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int NB = layer->N / 64, KB = layer->K / 128;
+}  // extern "C"
 
+namespace {
+
+// One token on a layer whose runs hold at most two blocks on average: the
+// decode kernel builds its activation records itself (no prologue kernel, one
+// launch boundary less on this latency-bound path).
+bool fused_one_token(const mpq_layer* layer, int32_t M) {
+    const size_t blocks = (size_t)(layer->N / 64) * (layer->K / 128);
+    return M == 1 && blocks <= 2 * (size_t)layer->n_units;
+}
+
+// Decode-kernel arguments of one layer (the token group is set by the caller).
+DecodeParams decode_params(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
+                           const LinearWs& w) {
+    DecodeParams dp{};
+    dp.codes = static_cast<const uint8_t*>(layer->codes);
+    dp.desc = layer->sched;
+    dp.bits8 = reinterpret_cast<const uint8_t*>(layer->sched + (size_t)layer->n_units * DESC_WORDS);
+    dp.scales = layer->scales;
+    dp.zeros = layer->zeros;
+    dp.row_perm = layer->row_perm;
+    dp.xq = reinterpret_cast<const uint8_t*>(w.xq);
+    dp.x = static_cast<const uint16_t*>(x_dev);
+    dp.col_perm = layer->col_perm;
+    dp.y = y_dev;
+    dp.partial = w.partial;
+    dp.counters = w.counters;
+    dp.err = w.err;
+    dp.N = layer->N;
+    dp.K = layer->K;
+    dp.NB = layer->N / 64;
+    dp.KB = layer->K / 128;
+    dp.M_total = M;
+    dp.n_units = layer->n_units;
+    dp.m0 = 0;
+    dp.Mg = 1;
+    return dp;
+}
+
+// mpq_linear on a carved workspace (arguments already checked).
+mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
+                      const LinearWs& w, cudaStream_t s, void* ev_begin, void* ev_end) {
+    const int NB = layer->N / 64, KB = layer->K / 128;
     const bool use_tc = M > kDecodeMaxM;
     if (!use_tc && (uint64_t)KB * (uint64_t)M * XQD_REC >= (1ull << 32)) return MPQ_ERR_SHAPE;
-    // one token on a layer whose runs hold at most two blocks on average: the
-    // decode kernel builds its activation records itself (no prologue kernel,
-    // one launch boundary less on this latency-bound path)
-    const bool fused = !use_tc && M == 1 && (size_t)NB * KB <= 2 * (size_t)layer->n_units;
+    const bool fused = !use_tc && fused_one_token(layer, M);
     XprepParams xp{};
     xp.x = static_cast<const uint16_t*>(x_dev);
     xp.col_perm = layer->col_perm;
@@ -581,26 +609,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     if (e == cudaSuccess) e = ensure_smem_attr(k_decode<false>, (int)sizeof(DecSmem), g_decode_attr8);
     if (e == cudaSuccess) e = ensure_smem_attr(k_decode<true, true>, (int)sizeof(DecSmem), g_decode_attr_f);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
-    DecodeParams dp{};
-    dp.codes = static_cast<const uint8_t*>(layer->codes);
-    dp.desc = layer->sched;
-    dp.bits8 = reinterpret_cast<const uint8_t*>(layer->sched + (size_t)layer->n_units * DESC_WORDS);
-    dp.scales = layer->scales;
-    dp.zeros = layer->zeros;
-    dp.row_perm = layer->row_perm;
-    dp.xq = reinterpret_cast<const uint8_t*>(w.xq);
-    dp.x = static_cast<const uint16_t*>(x_dev);
-    dp.col_perm = layer->col_perm;
-    dp.y = y_dev;
-    dp.partial = w.partial;
-    dp.counters = w.counters;
-    dp.err = w.err;
-    dp.N = layer->N;
-    dp.K = layer->K;
-    dp.NB = NB;
-    dp.KB = KB;
-    dp.M_total = M;
-    dp.n_units = layer->n_units;
+    DecodeParams dp = decode_params(layer, x_dev, M, y_dev, w);
 
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)((layer->n_units + DEC_WARPS - 1) / DEC_WARPS));
@@ -625,6 +634,87 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
         return MPQ_ERR_CUDA;
     return MPQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
+                            void* ws, size_t ws_bytes, void* stream, void* ev_begin,
+                            void* ev_end) {
+    mpq_status st = check_layer(layer);
+    if (st != MPQ_OK) return st;
+    if (M < 0) return MPQ_ERR_SHAPE;
+    if (M == 0) return MPQ_OK;
+    if (!x_dev || !y_dev) return MPQ_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
+    LinearWs w = carve_linear(ws, layer, M);
+    if (ws_bytes < w.bytes) return MPQ_ERR_WORKSPACE;
+    return linear_run(layer, x_dev, M, y_dev, w, static_cast<cudaStream_t>(stream), ev_begin, ev_end);
+}
+
+size_t mpq_linear_group_workspace_size(const mpq_layer* layers, int32_t n, int32_t M) {
+    if (!layers || n < 1 || n > MPQ_GROUP_MAX || M < 0) return 0;
+    size_t total = 0;
+    for (int i = 0; i < n; ++i) total += round256(carve_linear(nullptr, &layers[i], M).bytes);
+    return total;
+}
+
+mpq_status mpq_linear_group(const mpq_layer* layers, int32_t n, const void* x_dev, int32_t M,
+                            float* const* y_devs, void* ws, size_t ws_bytes, void* stream) {
+    if (!layers || !y_devs || n < 1 || n > MPQ_GROUP_MAX) return MPQ_ERR_ARG;
+    for (int i = 0; i < n; ++i) {
+        const mpq_status st = check_layer(&layers[i]);
+        if (st != MPQ_OK) return st;
+        if (layers[i].K != layers[0].K) return MPQ_ERR_SHAPE;
+        if (!y_devs[i]) return MPQ_ERR_ARG;
+    }
+    if (M < 0) return MPQ_ERR_SHAPE;
+    if (M == 0) return MPQ_OK;
+    if (!x_dev) return MPQ_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
+    if (ws_bytes < mpq_linear_group_workspace_size(layers, n, M)) return MPQ_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // each layer's part of the workspace; one error word (the first) for all
+    static_assert(MPQ_GROUP_MAX == DEC_GROUP_MAX, "group size of the C ABI and the kernel");
+    LinearWs w[MPQ_GROUP_MAX];
+    size_t off = 0;
+    bool all_fused = true;
+    for (int i = 0; i < n; ++i) {
+        w[i] = carve_linear(static_cast<uint8_t*>(ws) + off, &layers[i], M);
+        w[i].err = static_cast<uint32_t*>(ws);
+        off += round256(w[i].bytes);
+        all_fused = all_fused && fused_one_token(&layers[i], M);
+    }
+    if (!all_fused) {
+        for (int i = 0; i < n; ++i) {
+            const mpq_status st = linear_run(&layers[i], x_dev, M, y_devs[i], w[i], s, nullptr, nullptr);
+            if (st != MPQ_OK) return st;
+        }
+        return MPQ_OK;
+    }
+    // one launch over all the layers' runs
+    cudaError_t e = ensure_smem_attr(k_decode_group, (int)sizeof(DecSmem), g_decode_attr_g);
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    DecodeGroup gp{};
+    gp.n = n;
+    gp.unit_begin[0] = 0;
+    for (int i = 0; i < n; ++i) {
+        gp.layer[i] = decode_params(&layers[i], x_dev, M, y_devs[i], w[i]);
+        gp.unit_begin[i + 1] = gp.unit_begin[i] + layers[i].n_units;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((gp.unit_begin[n] + DEC_WARPS - 1) / DEC_WARPS));
+    cfg.blockDim = dim3(DEC_THREADS);
+    cfg.dynamicSmemBytes = sizeof(DecSmem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, k_decode_group, gp));
 }
 
 size_t mpq_linear_host_workspace_size(const mpq_layer* layer, int32_t M) {

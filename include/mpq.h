@@ -212,6 +212,26 @@ mpq_status mpq_linear_typed(const mpq_layer* layer, const void* x_dev, int32_t M
                             void* y_dev, mpq_ydtype ydt, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* Several layers that share x (the same K): y_i = x * dequant(W_i)^T for
+ * i < n, e.g. the q, k and v projections or gate and up.  Same results as n
+ * mpq_linear calls (bit for bit); when M == 1 and every layer's decode
+ * builds its own activation records (layers whose runs hold at most two
+ * blocks on average), the whole group is one kernel launch -- the launch
+ * floor, which dominates such small layers, is paid once per group instead
+ * of once per layer (the pages have no grouped call; this is a deployment
+ * convenience of the library).  Otherwise the layers run one after another.
+ *   layers  host array of n layers (1 <= n <= MPQ_GROUP_MAX), equal K.
+ *   y_devs  host array of n device pointers (fp32, M x N_i each).
+ *   ws      device workspace of mpq_linear_group_workspace_size(layers, n, M)
+ *           bytes, 256-byte aligned, zero-filled before first use (as for
+ *           mpq_linear); its first word is the group's error word.
+ * Host errors: ARG (n out of range, NULL), SHAPE (K differs, bad layer),
+ * WORKSPACE; device (mpq_check): TIMEOUT. */
+#define MPQ_GROUP_MAX 8
+size_t mpq_linear_group_workspace_size(const mpq_layer* layers, int32_t n, int32_t M);
+mpq_status mpq_linear_group(const mpq_layer* layers, int32_t n, const void* x_dev, int32_t M,
+                            float* const* y_devs, void* ws, size_t ws_bytes, void* stream);
+
 /* mpq_linear that also records two CUDA events (cudaEvent_t as void*; either
  * may be NULL) on `stream`: ev_begin right before the first launch of the
  * main GEMM kernel and ev_end right after its last launch, so a caller can

@@ -130,3 +130,30 @@ def test_linear_typed_host_validation(lib):
     assert B.STATUS[typed(ctypes.byref(layer), P(16), M, None, B.Y_BF16, P(256), b16,
                           None)] == "MPQ_ERR_ARG"
     assert typed(ctypes.byref(layer), P(16), 0, P(16), B.Y_BF16, P(256), b16, None) == 0
+
+
+def test_linear_group_host_validation(lib):
+    """mpq_linear_group: sizes add up layer by layer; bad groups are refused
+    before any launch."""
+    La = B.plan(128, 256, np.array([1, 2, 3, 4], np.uint8))
+    Lb = B.plan(64, 256, np.array([2, 0], np.uint8))
+    Lc = B.plan(64, 512, np.array([2, 0, 1, 1], np.uint8))
+    a, b, c = _fake_layer(La), _fake_layer(Lb), _fake_layer(Lc)
+    P = ctypes.c_void_p
+    M = 1
+    arr = (B.Layer * 2)(a, b)
+    need = lib.mpq_linear_group_workspace_size(arr, 2, M)
+    each = [lib.mpq_linear_workspace_size(ctypes.byref(l), M) for l in (a, b)]
+    assert need == sum((e + 255) // 256 * 256 for e in each)
+    ys = (ctypes.c_void_p * 2)(16, 16)
+    grp = lib.mpq_linear_group
+    assert B.STATUS[grp(arr, 0, P(16), M, ys, P(256), need, None)] == "MPQ_ERR_ARG"
+    assert B.STATUS[grp(arr, 9, P(16), M, ys, P(256), need, None)] == "MPQ_ERR_ARG"
+    assert B.STATUS[grp(arr, 2, P(16), M, ys, P(256), need - 1, None)] == "MPQ_ERR_WORKSPACE"
+    assert B.STATUS[grp(arr, 2, None, M, ys, P(256), need, None)] == "MPQ_ERR_ARG"
+    assert B.STATUS[grp(arr, 2, P(16), M, (ctypes.c_void_p * 2)(16, None), P(256), need,
+                        None)] == "MPQ_ERR_ARG"
+    mixed = (B.Layer * 2)(a, c)   # K 256 and 512
+    assert B.STATUS[grp(mixed, 2, P(16), M, ys, P(256), 1 << 20, None)] == "MPQ_ERR_SHAPE"
+    assert grp(arr, 2, P(16), 0, ys, P(256), need, None) == 0
+    assert lib.mpq_linear_group_workspace_size(arr, 9, M) == 0

@@ -317,3 +317,37 @@ def test_workspace_reuse(mpq):
         torch.cuda.synchronize()
         assert torch.equal(got, want), i
     assert _lib.lib().mpq_check(ws.data_ptr(), None) == 0
+
+
+@pytest.mark.parametrize("M", [1, 3, 40])
+def test_linear_group(mpq, oracle, M):
+    """mpq_linear_group equals one mpq_linear per layer bit for bit: one launch
+    for short-run layers at M == 1, the layers one after another otherwise;
+    and each output meets the oracle's bounds."""
+    import torch
+    specs = [("q", 1024, 1024, 2.1, "saliency"), ("k", 256, 1024, 2.5, "random"),
+             ("v", 512, 1024, 3.0, "random")]
+    Ls = [synth.make_layer(n, N, K, b, 7000 + i, perm) for i, (n, N, K, b, perm) in enumerate(specs)]
+    Ps = [pack_gpu(mpq, L) for L in Ls]
+    x_bits = synth.make_x(7100 + M, M, 1024)
+    x = dev(x_bits)
+    ys = mpq.linear_group(Ps, x)
+    torch.cuda.synchronize()
+    for L, P, y in zip(Ls, Ps, ys):
+        assert torch.equal(y, mpq.linear(P, x))
+        R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+        y_ref, bnd = oracle.linear(R, x_bits)
+        assert_y_close(y.cpu().numpy(), y_ref, bnd)
+
+
+def test_linear_group_mixed_runs(mpq):
+    """A group with a long-run layer (its decode needs the prologue kernel)
+    runs layer by layer and still equals the single calls."""
+    import torch
+    big = synth.config_layer(3, 0)                 # 14336 x 4096, ~3 blocks per run
+    small = synth.config_layer(2, 0)               # 4096 x 4096, one block per run
+    Ps = [pack_gpu(mpq, big), pack_gpu(mpq, small)]
+    x = dev(synth.make_x(7200, 1, 4096))
+    ys = mpq.linear_group(Ps, x)
+    for P, y in zip(Ps, ys):
+        assert torch.equal(y, mpq.linear(P, x))
