@@ -2,7 +2,9 @@
 // larger token counts.
 //
 // D[i][m] = sum_k w_hat'[i][k] * x'[m][k] for a tile of 128 weight rows
-// (two 64-row block rows) and 128 tokens; y[m][row_perm[i]] = D * tok_scale[m].
+// (two 64-row block rows) and BN = 128 or 256 tokens, over all k blocks or
+// one split of them; y[m][row_perm[i]] = D * tok_scale[m] (the splits summed
+// and the rows reordered by k_finish_rows).
 // The blocks' dequantization is the RTN of the ScaleBITS summary ("Approach",
 // "Key results"); TileQuant's abstract describes the same split -- compact
 // per-tile buffers expanded next to the 16-bit tensor-core computation.
@@ -19,7 +21,7 @@
 //              into the K-major 128B-swizzled shared-memory A operand (four
 //              warps per TMEM lane quadrant keep the schedulers busy); after
 //              the last k block they read the fp32 accumulator out of TMEM
-//              and write y.
+//              and write y' in W' row order (or the split's partial sums).
 // A k block whose two blocks are both 0-bit is skipped by every role (no
 // bytes, no MMA); a 0-bit block next to a non-zero one contributes zero rows.
 // The operands are fp16 (A = dequantized weights, B = x' scaled per token by a

@@ -796,8 +796,9 @@ mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t
         }
         scratch = g_noalloc_ptr[dev];
     }
-    // The existing path clears the scratch's error word and fix-up counters
-    // (the only parts that must start at zero) at the start of every call.
+    // The scratch starts zeroed (static storage) and every call that ends
+    // without a device error leaves its counters at zero; the error word
+    // keeps the first device error.
     return mpq_linear(layer, x_dev, M, y_dev, scratch, (size_t)MPQ_NOALLOC_SCRATCH_BYTES, stream);
 }
 
