@@ -214,7 +214,8 @@ def test_linear_host_entry_point(mpq, oracle):
 # sampled output rows the oracle computes one by one.
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("cfg,proj,Ms", [(3, 0, (1, 8, 16, 32)), (3, 2, (1, 8)),
-                                         (4, 1, (1, 4, 16)), (4, 3, (1,)),
+                                         (4, 0, (1, 4, 16)), (4, 1, (1, 4, 16)), (4, 3, (1,)),
+                                         (4, 4, (1,)), (4, 6, (1,)),
                                          # tensor-core path at the prefill sizes, 256-token
                                          # tiles: k split in 2 (q at 512), in 4 (k at ragged
                                          # 700), not split (2048, down at ragged 1100)
