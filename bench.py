@@ -621,8 +621,6 @@ def run_reference(args):
     for _ in range(args.steps):
         oracle.linear_rows(R, x, rows)
     el = time.perf_counter() - t0
-    if prev is not None:
-        oracle.set_threads(prev)
     frac = len(rows) / layer.N
     T = (layer.N // 64) * (layer.K // 128)
     nbytes = algorithmic_bytes(layer.N, layer.K, M, R.codes.size * frac, R.scales.size * frac,
