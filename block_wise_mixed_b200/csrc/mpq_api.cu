@@ -245,10 +245,19 @@ LinearWs carve_linear(void* ws, const mpq_layer* layer, int32_t M) {
     return w;
 }
 
+// The kernels read the layer's buffers with 16-byte vector loads and bulk
+// copies, which need 16-byte aligned addresses.
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool layer_aligned(const mpq_layer* L) {
+    return aligned16(L->codes) && aligned16(L->table) && aligned16(L->sched) && aligned16(L->scales) &&
+           aligned16(L->zeros) && aligned16(L->row_perm) && aligned16(L->col_perm);
+}
+
 mpq_status check_layer(const mpq_layer* L) {
     if (!L) return MPQ_ERR_ARG;
     if (L->N <= 0 || L->K <= 0 || L->N % 64 || L->K % 128) return MPQ_ERR_SHAPE;
     if (!L->table || !L->sched || L->n_units <= 0) return MPQ_ERR_ARG;
+    if (!layer_aligned(L)) return MPQ_ERR_ARG;
     return MPQ_OK;
 }
 
@@ -357,6 +366,7 @@ mpq_status mpq_pack_timed(const mpq_layout* L, const void* W_dev, const uint8_t*
     if (!out->table || !out->sched || (L->codes_bytes && !out->codes) ||
         (L->n_sz && (!out->scales || !out->zeros)))
         return MPQ_ERR_ARG;
+    if (!layer_aligned(out) || !aligned16(W_dev)) return MPQ_ERR_ARG;
     if (!ws || ws_bytes < mpq_pack_workspace_size(L)) return MPQ_ERR_WORKSPACE;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -432,7 +442,7 @@ mpq_status mpq_linear_typed(const mpq_layer* layer, const void* x_dev, int32_t M
     if (st != MPQ_OK) return st;
     if (M < 0) return MPQ_ERR_SHAPE;
     if (M == 0) return MPQ_OK;
-    if (!x_dev || !y_dev) return MPQ_ERR_ARG;
+    if (!x_dev || !y_dev || !aligned16(x_dev)) return MPQ_ERR_ARG;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
     const size_t base = round256(carve_linear(nullptr, layer, M).bytes);
     const size_t n = (size_t)M * layer->N;
@@ -647,7 +657,7 @@ mpq_status mpq_linear_timed(const mpq_layer* layer, const void* x_dev, int32_t M
     if (st != MPQ_OK) return st;
     if (M < 0) return MPQ_ERR_SHAPE;
     if (M == 0) return MPQ_OK;
-    if (!x_dev || !y_dev) return MPQ_ERR_ARG;
+    if (!x_dev || !y_dev || !aligned16(x_dev)) return MPQ_ERR_ARG;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
     LinearWs w = carve_linear(ws, layer, M);
     if (ws_bytes < w.bytes) return MPQ_ERR_WORKSPACE;
@@ -672,7 +682,7 @@ mpq_status mpq_linear_group(const mpq_layer* layers, int32_t n, const void* x_de
     }
     if (M < 0) return MPQ_ERR_SHAPE;
     if (M == 0) return MPQ_OK;
-    if (!x_dev) return MPQ_ERR_ARG;
+    if (!x_dev || !aligned16(x_dev)) return MPQ_ERR_ARG;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return MPQ_ERR_WORKSPACE;
     if (ws_bytes < mpq_linear_group_workspace_size(layers, n, M)) return MPQ_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -64,6 +64,9 @@
  *     the workspace was zero-filled or since the last mpq_check(), which
  *     reports and clears it (mpq_pack clears it when it starts).
  *   - A launch failure returns MPQ_ERR_CUDA.
+ *   - Every device pointer that the kernels read -- W, x, and the codes,
+ *     table, sched, scales, zeros and permutations of a layer -- must be
+ *     16-byte aligned (vector loads and bulk copies); MPQ_ERR_ARG otherwise.
  *   - Limits: N % 64 == 0, K % 128 == 0, N, K > 0, K <= 65536 when a column
  *     permutation is given, codes_bytes < 2^32; M >= 0 (M == 0 is a no-op).
  */

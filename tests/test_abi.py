@@ -157,3 +157,30 @@ def test_linear_group_host_validation(lib):
     assert B.STATUS[grp(mixed, 2, P(16), M, ys, P(256), 1 << 20, None)] == "MPQ_ERR_SHAPE"
     assert grp(arr, 2, P(16), 0, ys, P(256), need, None) == 0
     assert lib.mpq_linear_group_workspace_size(arr, 9, M) == 0
+
+
+@pytest.mark.parametrize("field", ["codes", "table", "sched", "scales", "zeros", "row_perm", "col_perm"])
+def test_misaligned_layer_pointers_refused(lib, field):
+    """Every buffer the kernels read with vector loads or bulk copies must be
+    16-byte aligned; a misaligned one is refused before any launch."""
+    L = B.plan(128, 256, np.array([1, 2, 3, 4], np.uint8))
+    layer = _fake_layer(L, rp=True, cp=True)
+    P = ctypes.c_void_p
+    need = lib.mpq_linear_workspace_size(ctypes.byref(layer), 4)
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), P(16), 0, P(16), P(256), need, None)] == "MPQ_OK"
+    setattr(layer, field, 24)
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), P(16), 4, P(16), P(256), need, None)] == "MPQ_ERR_ARG"
+
+
+def test_misaligned_x_and_w_refused(lib):
+    L = B.plan(128, 256, np.array([1, 2, 3, 4], np.uint8))
+    layer = _fake_layer(L)
+    P = ctypes.c_void_p
+    need = lib.mpq_linear_workspace_size(ctypes.byref(layer), 4)
+    assert B.STATUS[lib.mpq_linear(ctypes.byref(layer), P(18), 4, P(16), P(256), need, None)] == "MPQ_ERR_ARG"
+    bits = np.array([1, 2, 3, 4], np.uint8)
+    out = _fake_layer(L)
+    ws_need = lib.mpq_pack_workspace_size(ctypes.byref(L))
+    st = lib.mpq_pack(ctypes.byref(L), P(8), bits.ctypes.data_as(P), None, None, ctypes.byref(out),
+                      P(256), ws_need, None)
+    assert B.STATUS[st] == "MPQ_ERR_ARG"
