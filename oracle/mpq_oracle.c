@@ -25,7 +25,7 @@
  *             Mixed-Precision Post-Training Quantization", abstract: the
  *             precision map guides the layout of compact weight buffers.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *   - a block is 64 output rows x 128 input columns, so each block row is one
  *     quantization group of 128 weights;
  *   - RTN is asymmetric with the range widened to include 0; the fp16 scale is
