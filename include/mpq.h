@@ -55,8 +55,10 @@
  *
  * Conventions:
  *   - The caller owns every buffer.  The library allocates no device memory
- *     and keeps no global state; calls are asynchronous on `stream` (a
- *     cudaStream_t passed as void*; NULL = the legacy default stream).
+ *     and keeps no state between calls beyond one-time kernel attributes per
+ *     device (and mpq_linear_noalloc's static scratch, below); calls are
+ *     asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream).
  *   - Errors that the host can see are returned at once and nothing is
  *     launched.  Errors found in device data (non-finite W, a group with no
  *     representable scale) or a device wait that ran out are written to an
