@@ -91,6 +91,8 @@ def lib():
         L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
         L.mpq_linear_noalloc.argtypes = [ctypes.POINTER(Layer), P, i32, P, P]
         L.mpq_linear_noalloc.restype = ctypes.c_int
+        L.mpq_noalloc_check.argtypes = [P]
+        L.mpq_noalloc_check.restype = ctypes.c_int
         L.mpq_check.argtypes = [P, P]
         L.mpq_status_string.argtypes = [ctypes.c_int]
         L.mpq_status_string.restype = ctypes.c_char_p

@@ -8,7 +8,6 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
-#include <mutex>
 #include <vector>
 
 #include "../../include/mpq.h"
@@ -772,14 +771,19 @@ mpq_status mpq_check(const void* ws, void* stream) {
 // memory.  Its scratch is this fixed array, which every device that loads the
 // library holds until the process exits.  Host code must not hand the
 // array's name to a kernel (in host code it is only a stand-in for the
-// symbol); the device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call there.
+// symbol); the device address is looked up with cudaGetSymbolAddress, with
+// the calling device current, on every call (the lookup allocates nothing,
+// and a fresh lookup stays right after the device's context is recreated).
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MPQ_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
+mpq_status noalloc_scratch(void** out) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MPQ_ERR_CUDA;
+    *out = p;
+    return MPQ_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -792,24 +796,28 @@ mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t
     if (M == 0) return MPQ_OK;
     if (mpq_linear_workspace_size(layer, M) > (size_t)MPQ_NOALLOC_SCRATCH_BYTES)
         return MPQ_ERR_WORKSPACE;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MPQ_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return MPQ_ERR_ARG;
     void* scratch = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
-            void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
-                return MPQ_ERR_CUDA;
-            g_noalloc_ptr[dev] = p;
-        }
-        scratch = g_noalloc_ptr[dev];
-    }
+    st = noalloc_scratch(&scratch);
+    if (st != MPQ_OK) return st;
     // The scratch starts zeroed (static storage) and every call that ends
     // without a device error leaves its counters at zero; the error word
-    // keeps the first device error.
+    // keeps the first device error until mpq_noalloc_check reads it.
     return mpq_linear(layer, x_dev, M, y_dev, scratch, (size_t)MPQ_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+mpq_status mpq_noalloc_check(void* stream) {
+    void* scratch = nullptr;
+    mpq_status st = noalloc_scratch(&scratch);
+    if (st != MPQ_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t err = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MPQ_ERR_CUDA;
+    if (cudaMemcpy(&err, scratch, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MPQ_ERR_CUDA;
+    // A call that stopped on a device error may have left arrival counters
+    // set: clear the whole array, back to its state at load time.
+    if (err != 0u && cudaMemset(scratch, 0, (size_t)MPQ_NOALLOC_SCRATCH_BYTES) != cudaSuccess)
+        return MPQ_ERR_CUDA;
+    return static_cast<mpq_status>(err);
 }
 
 const char* mpq_status_string(mpq_status s) {

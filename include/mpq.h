@@ -268,18 +268,28 @@ mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host,
  *   until the process exits; no cudaMalloc/cudaFree or other allocating
  *   call is made.  Sizes whose workspace (mpq_linear_workspace_size) would
  *   exceed it return MPQ_ERR_WORKSPACE.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   Every call looks up the array's device address (cudaGetSymbolAddress)
+ *   with the calling device current; the first lookup on a device loads the
+ *   library's device code there, so make the first call before any stream
+ *   capture.
  *   All calls share the one array, which starts zeroed and keeps the last
  *   call's contents (the parts that must start at zero are left at zero): calls
  *   that overlap on the GPU -- on different streams, or from different
  *   threads -- race and give wrong results.  Serialize them.
- *   Device-side errors go to the array's error word, which mpq_check cannot
- *   see; host-side errors are returned as for mpq_linear. */
+ *   Device-side errors (MPQ_ERR_TIMEOUT) go to the array's error word, which
+ *   mpq_check cannot see: read it with mpq_noalloc_check.  Until then, a call
+ *   that stopped on a device error may have left the array's counters set,
+ *   and the calls after it give wrong results.  Host-side errors are returned
+ *   as for mpq_linear. */
 #define MPQ_NOALLOC_SCRATCH_BYTES (6u << 20)
 mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t M,
                               float* y_dev, void* stream);
+
+/* The error word of mpq_linear_noalloc's static array on the current device:
+ * synchronizes `stream`, returns the first device error of the calls since
+ * the previous check (MPQ_OK if none) and, after an error, zero-fills the
+ * array (memset, no allocation) so that the next call starts clean. */
+mpq_status mpq_noalloc_check(void* stream);
 
 /* Synchronizes `stream` and returns the device error word of `ws`: the first
  * device error of the mpq_linear calls on that workspace since it was

@@ -56,8 +56,10 @@ def _json_lines(text):
 
 
 def test_reference_arm_line():
+    # the 4096x4096 workload's layer keeps the CPU suite short; the arm's
+    # default is the 70B decoder layer
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
-                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+                        "--warmup", "3", "--cfg", "2"], cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
@@ -72,7 +74,7 @@ def test_reference_arm_two_ranks():
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
-           "reference", "--gpus", "2", "--steps", "2", "--warmup", "3"]
+           "reference", "--gpus", "2", "--steps", "2", "--warmup", "3", "--cfg", "2"]
     r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)

@@ -83,8 +83,9 @@ def test_pack_bit_exact_configs(mpq, oracle, cfg):
     check_sched(P, L.bits)
 
 
-@pytest.mark.parametrize("cfg,M", [(1, 1), (1, 2), (1, 3), (1, 7), (1, 8), (1, 9), (1, 17),
-                                   (1, 33), (2, 1), (2, 4), (2, 8)])
+@pytest.mark.parametrize("cfg,M", [(1, 1), (1, 2), (1, 3), (1, 7), (1, 8), (1, 9), (1, 16),
+                                   (1, 17), (1, 31), (1, 32), (1, 33), (1, 63), (1, 64),
+                                   (1, 65), (2, 1), (2, 4), (2, 8), (2, 16)])
 def test_linear_configs(mpq, oracle, cfg, M):
     L = synth.config_layer(cfg, 0)
     P = pack_gpu(mpq, L)
@@ -213,21 +214,49 @@ def test_linear_host_entry_point(mpq, oracle):
 # Full-size layers in the benchmark's launch configuration, checked on
 # sampled output rows the oracle computes one by one.
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("cfg,proj,Ms", [(3, 0, (1, 8, 16, 32)), (3, 2, (1, 8)),
-                                         (4, 0, (1, 4, 16)), (4, 1, (1, 4, 16)), (4, 3, (1,)),
-                                         (4, 4, (1,)), (4, 6, (1,)),
-                                         # tensor-core path at the prefill sizes, 256-token
-                                         # tiles: k split in 2 (q at 512), in 4 (k at ragged
-                                         # 700), not split (2048, down at ragged 1100)
-                                         (5, 0, (512, 2048)), (5, 1, (700,)), (5, 6, (1100,))])
+# Every projection of the three large workloads at every batch size they
+# name: the Llama-3-8B MLP (gate, up, down) at M = 1, 8, 16, 32; the
+# Llama-3-70B decoder layer (q, k, v, o, gate, up, down) at M = 1, 4, 16; the
+# Llama-3-8B layer on the tensor-core path at M = 512 and 2048; plus ragged
+# tensor-core batches (k at 700: k split in 4; down at 1100: not split).
+FULL_CELLS = ([(3, p, (1, 8, 16, 32)) for p in range(3)] +
+              [(4, p, (1, 4, 16)) for p in range(7)] +
+              [(5, p, (512, 2048)) for p in range(7)] +
+              [(5, 1, (700,)), (5, 6, (1100,))])
+
+
+def sampled_rows(P, L, seed, n_random=96):
+    """Output rows to check: random ones plus every row of the block rows that
+    several decode runs share (their sums are finished by the last arriving
+    run), mapped through the row order."""
+    from block_wise_mixed_b200 import _lib
+    lay = P.layout
+    sched = _lib.plan_schedule(lay, L.bits)
+    desc = sched[:lay.n_units * 32].reshape(-1, 32)
+    t0, t1 = desc[:, 0].astype(np.int64), desc[:, 1].astype(np.int64)
+    first, last = t0 // lay.KB, (t1 - 1) // lay.KB
+    shared = set()
+    for nb in np.unique(np.concatenate([first, last])):
+        if int(np.sum((first <= nb) & (last >= nb))) > 1:
+            shared.add(int(nb))
+    shared = sorted(shared)
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(len(shared), min(len(shared), 6), replace=False) if shared else []
+    rows_p = [64 * shared[i] + r for i in pick for r in (0, 1, 31, 62, 63)]
+    rows_p = np.array(rows_p, dtype=np.int64)
+    rows = L.row_perm[rows_p] if L.row_perm is not None else rows_p
+    rows = np.concatenate([rows, rng.choice(L.N, n_random, replace=False)])
+    return np.unique(rows).astype(np.int32)
+
+
+@pytest.mark.parametrize("cfg,proj,Ms", FULL_CELLS)
 def test_full_size_sampled(mpq, oracle, cfg, proj, Ms):
     L = synth.config_layer(cfg, proj)
     P = pack_gpu(mpq, L)
     R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
     assert_pack_equal(P, R)
     check_sched(P, L.bits)
-    rng = np.random.default_rng(cfg * 10 + proj)
-    rows = np.sort(rng.choice(L.N, 96, replace=False)).astype(np.int32)
+    rows = sampled_rows(P, L, cfg * 10 + proj)
     for M in Ms:
         x = synth.make_x(synth.seed_of(cfg, proj), M, L.K)
         y = run_linear(mpq, P, x)

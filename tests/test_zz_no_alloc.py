@@ -32,12 +32,25 @@ def _noalloc(lib, P, x, y):
                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("cfg,M", [(1, 1), (1, 5), (2, 1), (2, 8)])
-def test_noalloc_matches_workspace_entry_point(mpq, oracle, cfg, M):
+def _layer(spec):
+    if spec[0] == "cfg":
+        return synth.config_layer(spec[1], 0)
+    _, N, K = spec      # a tensor-core shape whose k blocks are split across CTAs
+    return synth.make_layer("tc", N, K, 3.0, 4000 + N + K, "random")
+
+
+# Decode kernel (M <= 16) and tensor-core kernel (M > 16): the latter carves
+# its split-K partial sums out of the static array (N=512, K=128*11 at M=40
+# splits the k blocks in two) and reorders rows with a second kernel.
+@pytest.mark.parametrize("spec,M", [(("cfg", 1), 1), (("cfg", 1), 5), (("cfg", 2), 1),
+                                    (("cfg", 2), 8), (("cfg", 1), 33),
+                                    (("tc", 512, 128 * 11), 40)])
+def test_noalloc_matches_workspace_entry_point(mpq, oracle, spec, M):
     import torch
     from block_wise_mixed_b200 import _lib
     lib = _lib.lib()
-    L = synth.config_layer(cfg, 0)
+    L = _layer(spec)
+    cfg = spec[1] if spec[0] == "cfg" else 0
     P = mpq.pack(torch.from_numpy(L.W.view(np.int16)).cuda(), L.bits, L.row_perm, L.col_perm)
     R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
     for call in range(2):
@@ -55,6 +68,8 @@ def test_noalloc_matches_workspace_entry_point(mpq, oracle, cfg, M):
         assert np.all(np.abs(got - y_or) <= 1e-3 * bnd)
         assert np.linalg.norm(got - y_or) <= 5e-4 * np.linalg.norm(y_or)
         assert np.all(np.abs(got - ref) <= 1e-3 * bnd)
+    # no device error was recorded in the static array
+    assert lib.mpq_noalloc_check(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
 
 
 def test_noalloc_rejects_oversize(mpq):
