@@ -7,23 +7,29 @@
 //
 // Work split.  At pack time the blocks are cut into `n_units` row-major runs
 // of about equal estimated cost (bytes moved plus decode work per bit
-// width); each run is one warp's work.  A unit descriptor of 128 bytes holds
-// everything the warp needs to start: its run [t0, t1), the offsets of its
-// first block of every width in the code segments and in the scale/zero
-// arrays, the bit widths of its first 64 blocks, and where the partial sums
-// of its first and last block rows go.  One coalesced load of it is the only
-// dependent fetch before the first payload copy is issued.
+// width); each run is one warp's work.  A run descriptor of 128 bytes holds
+// its blocks [t0, t1), where its non-zero blocks start in the stage list and
+// how many there are, and where the partial sums of its first and last block
+// rows go.  The stage list holds, per non-zero block, everything its copies
+// need (payload offset, scale/zero index, block column and width, block
+// row): a warp loads 32 of them with one coalesced 16-byte load per lane.
 //
 // Each warp streams its non-zero blocks through a private ring of shared
 // memory with 1-D bulk async copies (payload + 64 scales + 64 zeros + the
-// activation slice in the column order of the block's low piece + F),
-// several blocks ahead of the one it computes.  Codes become exact fp16
-// subnormal pairs (q - z) * 2^-24 in registers (an AND or byte permute and
-// one HFMA2 per pair; the high piece of a split code is added in before the
-// multiply) and are multiplied on the tensor cores (mma.m16n8k16, fp32
-// accumulation).  Per block and output row: acc += s * F * c.  Forming
-// q - z per element keeps every product exact, so the fp32 rounding stays
-// relative to sum |x * w_hat| even when most codes equal the zero point.
+// activation record(s) of the block's slice), several blocks ahead of the
+// one it computes.
+//
+// Arithmetic (exact up to the final fp32 steps).  The activation slice is
+// held as integers X (k_xprep.cuh: X = rne(x' 2^e), |X| < 2^15, two s8
+// digits) and the codes as unsigned bytes: one AND of a code word gives four
+// codes of one "plane" (piece_regs).  The integer tensor cores
+// (mma.m16n8k32.u8.s8, s32 accumulation) form sum_j q_j X_j per digit with
+// no rounding, so the zero point can be taken out exactly:
+//   V = sum_j (q_j - z) X_j = C_l + 256 C_h - z T,   T = sum_j X_j,
+// and each block adds s * 2^-e * V to its output row in fp32.  The only
+// roundings are X (for slice elements more than 2^7 below the slice
+// maximum), the conversion of V to fp32 and the fp32 accumulation -- all
+// relative to sum |x * w_hat|, never to the cancelled sum q*x.
 //
 // A block row that lies inside one run is written straight to y.  A block
 // row shared by several runs (the first and last row of a run) is finished
@@ -41,25 +47,32 @@ namespace mpq {
 
 constexpr uint64_t DEC_WAIT_NS = 2000000000ull;
 
-// Unit descriptor: 32 words.
+// Run descriptor: 32 words (the unused ones are zero).
 enum DescWord {
-    DW_T0 = 0, DW_T1 = 1, DW_SZ = 2,
-    DW_CODE = 3,           // 3..9: code offset of the run's first block of width 1,2,3,4,5,6,8
+    DW_T0 = 0, DW_T1 = 1,  // the run's blocks [t0, t1)
+    DW_S0 = 2,             // index of its first non-zero block in the stage list
+    DW_NS = 3,             // number of non-zero blocks
     DW_A_SLOT = 10,        // first block row of the run: first partial slot of the row,
     DW_A_NC = 11,          //   number of runs that meet the row, this run's index among them
     DW_A_IDX = 12,
     DW_B_SLOT = 13,        // last block row of the run: the same three
     DW_B_NC = 14,
     DW_B_IDX = 15,
-    DW_BITS = 16,          // 16..31: bit widths of the run's first 64 blocks (bytes)
     DESC_WORDS = 32
 };
-constexpr int DESC_INLINE_BITS = 64;
+// Stage descriptor: one per non-zero block (block order), 4 words.
+enum StageWord {
+    SW_CODE = 0,           // byte offset of the payload in the codes buffer
+    SW_SZ = 1,             // index of the block's row 0 in scales / zeros
+    SW_KB_BITS = 2,        // block column | bit width << 16
+    SW_NB = 3,             // block row
+    STAGE_WORDS = 4
+};
 
 struct DecodeParams {
     const uint8_t* codes;
     const uint32_t* desc;     // [n_units][32]
-    const uint8_t* bits8;     // [NB*KB] bit width per block (runs longer than 64 blocks)
+    const uint4* stages;      // [non-zero blocks] stage descriptors
     const uint16_t* scales;
     const uint16_t* zeros;
     const int32_t* row_perm;
@@ -80,16 +93,15 @@ constexpr int DEC_WARPS = 4;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
 constexpr int DEC_CTAS_PER_SM = 4;   // 16 resident warps per SM
 constexpr int DEC_MAX_REGS = 112;
-constexpr int DEC_RING = 12288;      // bytes of ring per warp (>= largest stage)
+constexpr int DEC_RING = 12800;      // bytes of ring per warp (>= largest stage)
 constexpr int DEC_SLOTS = 8;         // stages in flight per warp
 constexpr int DEC_MAX_TOKENS = 8;
 
 struct DecWarp {
     uint8_t ring[DEC_RING];
-    int32_t rows[64];         // output index of each row of the current block row
-    __half xw[128];           // fused path: the block's x' slice, column order
+    int32_t rows[64];         // output index of each row of the current block row (16-byte aligned)
     uint64_t full[DEC_SLOTS];
-    uint4 zero16[4];          // zero B fragments for lanes beyond the token count
+    uint4 zero32[2];          // zero B fragments for lanes beyond the token count
 };
 struct DecSmem {
     DecWarp w[DEC_WARPS];
@@ -97,8 +109,9 @@ struct DecSmem {
 
 // DEC_CTAS_PER_SM x (smem + 1 KB reserved) must fit the SM's 228 KB
 static_assert(DEC_CTAS_PER_SM * (sizeof(DecSmem) + 1024) <= 228 * 1024, "decode smem too large");
-// largest stage: an 8-bit payload
+// largest stages: an 8-bit payload, or a 6-bit one with two activation variants
 static_assert(DEC_RING >= 8 * 1024 + 256 + DEC_MAX_TOKENS * XQD_VAR, "ring too small");
+static_assert(DEC_RING >= 6 * 1024 + 256 + 2 * DEC_MAX_TOKENS * XQD_VAR, "ring too small");
 
 __host__ __device__ constexpr int lo_width(int b) { return (b == 3) ? 2 : (b == 5 || b == 6) ? 4 : b; }
 __host__ __device__ constexpr int hi_width(int b) { return (b == 3 || b == 5) ? 1 : (b == 6) ? 2 : 0; }
@@ -107,199 +120,217 @@ __host__ __device__ constexpr int variant_of(int p) { return p == 1 ? 0 : p == 2
 __host__ __device__ constexpr int width_index(int b) { return b == 8 ? 6 : b - 1; }
 
 // ---------------------------------------------------------------------------
-// Code extraction.  For one row and the lane's 32 columns, a[pi] becomes the
-// fp16 pair ((q_a - z) * 2^-24, (q_b - z) * 2^-24) of pair pi (column order
-// of k_xprep.cuh) -- exact subnormals.  An AND (or byte permute) leaves a
-// code at bit `pos` of each half, i.e. the value q * 2^(pos-24); one HFMA2
-// with 2^-pos and zc = -z * 2^-24 gives (q - z) * 2^-24.  A split code adds
-// its high piece the same way, times 2^(low width), before the mma.
+// Code extraction.  piece_regs<P, W> turns this lane's quarter of one row of
+// a P-bit piece (columns 32t .. 32t+31 of the block) into the eight A-operand
+// registers of the four k-tiles of mma.m16n8k32 (index 2j + hf): four codes
+// per register, one per byte, each register one AND (and at most one shift)
+// of a code word -- a "plane" of the word.  The column that byte b of
+// register (j, hf) holds is xqd_col(variant of P, 32j + 16hf + 4t + b); the
+// activation records use the same order.  W shifts the codes left by W bits:
+// the high piece of a split code is worth 2^(low width) (3 = 2 + 1 bits,
+// 5 = 4 + 1, 6 = 4 + 2), so its planes carry that weight and both pieces
+// accumulate into the same sums (q = lo + 2^w(lo) hi <= 63 fits a byte).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ constexpr uint32_t h2pow(int k) {      // (2^k, 2^k) fp16 bits
-    return (uint32_t)((15 + k) << 10) * 0x10001u;
-}
-__device__ __forceinline__ uint32_t hadd2_bits(uint32_t a, uint32_t b) {
-    return h2_bits(__hadd2(bits_h2(a), bits_h2(b)));
+template <int S, int W>
+__device__ __forceinline__ uint32_t plane_shift(uint32_t w) {   // (w >> S) << W, as one shift
+    return (S >= W) ? (w >> (S - W)) : (w << (W - S));
 }
 
-template <int P>
-__device__ __forceinline__ void extract_lo(const uint32_t (&w)[P], uint32_t zc, uint32_t (&a)[16]) {
+template <int P, int W>
+__device__ __forceinline__ void piece_regs(const uint8_t* rowp, int t, uint32_t (&a)[8]) {
     if (P == 1) {
-        const uint32_t u = w[0], v = w[0] >> 8;
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            a[s] = hfma2_bits(u & (0x00010001u << s), h2pow(-s), zc);
-            a[8 + s] = hfma2_bits(v & (0x00010001u << s), h2pow(-s), zc);
-        }
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(rowp + 4 * t);
+        constexpr uint32_t m = 0x01010101u << W;
+        a[0] = plane_shift<0, W>(w) & m;
+        a[1] = plane_shift<1, W>(w) & m;
+        a[2] = plane_shift<2, W>(w) & m;
+        a[3] = plane_shift<3, W>(w) & m;
+        a[4] = plane_shift<4, W>(w) & m;
+        a[5] = plane_shift<5, W>(w) & m;
+        a[6] = plane_shift<6, W>(w) & m;
+        a[7] = plane_shift<7, W>(w) & m;
     } else if (P == 2) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const uint32_t u = w[i], v = w[i] >> 8;
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                a[8 * i + s] = hfma2_bits(u & (0x00030003u << (2 * s)), h2pow(-2 * s), zc);
-                a[8 * i + 4 + s] = hfma2_bits(v & (0x00030003u << (2 * s)), h2pow(-2 * s), zc);
-            }
-        }
+        const uint2 v = *reinterpret_cast<const uint2*>(rowp + 8 * t);
+        constexpr uint32_t m = 0x03030303u << W;
+        // register (j, hf): word j / 2, plane 2 (j % 2) + hf (bits 2 plane)
+        a[0] = plane_shift<0, W>(v.x) & m;
+        a[1] = plane_shift<2, W>(v.x) & m;
+        a[2] = plane_shift<4, W>(v.x) & m;
+        a[3] = plane_shift<6, W>(v.x) & m;
+        a[4] = plane_shift<0, W>(v.y) & m;
+        a[5] = plane_shift<2, W>(v.y) & m;
+        a[6] = plane_shift<4, W>(v.y) & m;
+        a[7] = plane_shift<6, W>(v.y) & m;
     } else if (P == 4) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t u = w[i], v = w[i] >> 8;
-            a[4 * i + 0] = hadd2_bits(u & 0x000F000Fu, zc);
-            a[4 * i + 1] = hfma2_bits(u & 0x00F000F0u, h2pow(-4), zc);
-            a[4 * i + 2] = hadd2_bits(v & 0x000F000Fu, zc);
-            a[4 * i + 3] = hfma2_bits(v & 0x00F000F0u, h2pow(-4), zc);
-        }
+        const uint4 v = *reinterpret_cast<const uint4*>(rowp + 16 * t);
+        a[0] = v.x & 0x0F0F0F0Fu; a[1] = (v.x >> 4) & 0x0F0F0F0Fu;
+        a[2] = v.y & 0x0F0F0F0Fu; a[3] = (v.y >> 4) & 0x0F0F0F0Fu;
+        a[4] = v.z & 0x0F0F0F0Fu; a[5] = (v.z >> 4) & 0x0F0F0F0Fu;
+        a[6] = v.w & 0x0F0F0F0Fu; a[7] = (v.w >> 4) & 0x0F0F0F0Fu;
     } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            a[2 * i + 0] = hadd2_bits(__byte_perm(w[i], 0u, 0x4240), zc);
-            a[2 * i + 1] = hadd2_bits(__byte_perm(w[i], 0u, 0x4341), zc);
-        }
+        const uint4 v0 = reinterpret_cast<const uint4*>(rowp + 32 * t)[0];
+        const uint4 v1 = reinterpret_cast<const uint4*>(rowp + 32 * t)[1];
+        a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
+        a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
     }
 }
 
-// High piece of a split code added onto the low pairs: a[pi] += 2^w * hi.
-// B = 3: low 2-bit, high 1-bit (w = 2); B = 5: 4 + 1 (w = 4); B = 6: 4 + 2.
-template <int B>
-__device__ __forceinline__ void add_hi(const uint32_t (&h)[B == 6 ? 2 : 1], uint32_t (&a)[16]) {
-    if (B == 3) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            // bytes 2i, 2i+1 hold the high bits of columns 16i..16i+7, 16i+8..16i+15
-            const uint32_t pb = __byte_perm(h[0], 0u, (2 * i) | (4 << 4) | ((2 * i + 1) << 8) | (4 << 12));
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                a[8 * i + s] = hfma2_bits(pb & (0x00010001u << s), h2pow(2 - s), a[8 * i + s]);
-                a[8 * i + 4 + s] = hfma2_bits(pb & (0x00010001u << (4 + s)), h2pow(-2 - s), a[8 * i + 4 + s]);
-            }
-        }
-    } else if (B == 5) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            // byte i holds the high bits of columns 8i..8i+7, in both halves
-            const uint32_t pb = __byte_perm(h[0], 0u, i | (4 << 4) | (i << 8) | (4 << 12));
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                // column 8i+r at bit r (low half), 8i+r+4 at bit r+4 (high half)
-                const uint32_t m = (uint32_t)((15 + 4 - r) << 10) | ((uint32_t)((15 - r) << 10) << 16);
-                a[4 * i + r] = hfma2_bits(pb & ((1u << r) | (1u << (20 + r))), m, a[4 * i + r]);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int b0 = 2 * (i & 1);
-            const uint32_t pb = __byte_perm(h[i >> 1], 0u, b0 | (4 << 4) | ((b0 + 1) << 8) | (4 << 12));
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-                a[4 * i + r] = hfma2_bits(pb & (0x00030003u << (2 * r)), h2pow(4 - 2 * r), a[4 * i + r]);
-        }
-    }
+// D(16x8, s32) += A(16x32, u8 codes) * B(32x8, s8 activation digits)
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int P>
-__device__ __forceinline__ void load_words(const uint8_t* p, uint32_t (&w)[P]) {
-    if (P == 1) {
-        w[0] = *reinterpret_cast<const uint32_t*>(p);
-    } else if (P == 2) {
-        const uint2 v = *reinterpret_cast<const uint2*>(p);
-        w[0] = v.x; w[1] = v.y;
-    } else if (P == 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(p);
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else {
-        const uint4 v0 = reinterpret_cast<const uint4*>(p)[0];
-        const uint4 v1 = reinterpret_cast<const uint4*>(p)[1];
-        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-        w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-    }
+__device__ __forceinline__ void load8(const uint8_t* src, uint32_t (&b)[8]) {
+    const uint4 v0 = reinterpret_cast<const uint4*>(src)[0];
+    const uint4 v1 = reinterpret_cast<const uint4*>(src)[1];
+    b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
+    b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
 }
 
-// One row's 16 pairs for width B (stage = payload; lane offset t).
-template <int B>
-__device__ __forceinline__ void row_pairs(const uint8_t* stage, int r, int t, uint32_t zc,
-                                          uint32_t (&a)[16]) {
+// One block of width B, added into acc.  The mma's rows are the block's rows
+// in an order that keeps each lane's rows together: in row tile rt, mma row
+// g is block row 8g + 2rt and mma row g + 8 is block row 8g + 2rt + 1 (two
+// adjacent rows: their scales and zero points are one fp16 pair).  mma
+// column 4u + d (d < 3) is digit d of token 2 grp + u; column 4u + 3 is zero.
+// Lane (g, t) accumulates columns 2t, 2t+1 -- digits (0, 1) of token
+// 2 grp + t/2 for even t, digit 2 for odd t -- of both rows; the lane pair
+// (t, t^1) swaps one partial sum so that the even lane finishes row
+// 8g + 2rt and the odd lane row 8g + 2rt + 1:
+//   V = (E_0 + 256 E_1) + 65536 E_2,  E_d = C_d - z T_d  (exact int32 parts)
+//   acc[rt][grp] += s * F * V        (lane row 8g + 2rt + (t & 1))
+template <int B, int G>
+__device__ __forceinline__ void block_accumulate(const uint8_t* stage, const uint8_t* xlo,
+                                                 const uint8_t* xhi, const uint8_t* zero32, int g,
+                                                 int t, uint32_t Mg, float (&acc)[4][G]) {
     constexpr int P0 = lo_width(B), P1 = hi_width(B);
-    uint32_t w[P0];
-    load_words<P0>(stage + r * 16 * P0 + t * 4 * P0, w);
-    extract_lo<P0>(w, zc, a);
-    if (P1) {
-        uint32_t h[B == 6 ? 2 : 1];
-        const uint8_t* hp = stage + 64 * 16 * P0 + r * 16 * P1 + t * 4 * P1;
-        if (B == 6) {
-            const uint2 v = *reinterpret_cast<const uint2*>(hp);
-            h[0] = v.x; h[B == 6 ? 1 : 0] = v.y;
-        } else {
-            h[0] = *reinterpret_cast<const uint32_t*>(hp);
-        }
-        add_hi<B>(h, a);
-    }
-}
-
-// One 16-row tile rt of a block of width B, added into acc:
-//   c = 2^-24 * sum over the block's 128 columns of (q - z) * x'
-//   acc[rt][*] += s_row * F_tok * c        (C-fragment order: rows 16rt+g,
-//   16rt+g+8 x tokens 2t, 2t+1).
-// The caller loops over rt at run time, so each width's code is one tile's
-// worth (small enough to stay in the instruction cache); the tile's eight
-// k-steps alternate between two accumulators to halve the mma chain.
-template <int B, bool ONE_TOKEN>
-__device__ __forceinline__ void tile_accumulate(const uint8_t* stage, const uint32_t (&b)[16], int rt,
-                                                int g, int t, float Fa, float Fb, float (&acc)[4][4]) {
-    const uint16_t* sc16 = reinterpret_cast<const uint16_t*>(stage + 1024 * B);
-    const int r0 = 16 * rt + g, r1 = r0 + 8;
-    // -z * 2^-24 in both halves (z is an fp16 integer; 0x8001 = -2^-24)
-    const uint32_t zc0 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)sc16[64 + r0], 0u, 0x1010)),
-                                         bits_h2(0x80018001u)));
-    const uint32_t zc1 = h2_bits(__hmul2(bits_h2(__byte_perm((uint32_t)sc16[64 + r1], 0u, 0x1010)),
-                                         bits_h2(0x80018001u)));
-    uint32_t a0[16], a1[16];
-    row_pairs<B>(stage, r0, t, zc0, a0);
-    row_pairs<B>(stage, r1, t, zc1, a1);
-    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint8_t* lo = stage;                       // 64 rows x 16 P0 bytes
+    const uint8_t* hi = stage + 64 * 16 * P0;        // 64 rows x 16 P1 bytes
+    const uint8_t* sz = stage + 1024 * B;            // scales[64], zeros[64] (fp16)
+    const bool odd = (t & 1) != 0;
+    // Four token groups: groups outermost, the codes unpacked again for each
+    // (fewer live registers); otherwise every group reuses a tile's codes.
+    constexpr bool kGroupOuter = G >= 4;
+    // B-fragment source of group grp: column g = token 2 grp + g/4, digit g%4
+    auto bsrc = [&](const uint8_t* x, int grp) -> const uint8_t* {
+        const uint32_t tb = 2u * grp + (uint32_t)(g >> 2), dg = (uint32_t)(g & 3);
+        return (dg < 3u && tb < Mg) ? x + tb * XQD_VAR + dg * 128 + t * 32 : zero32;
+    };
+    // digit sums and F of the lane's columns 2t, 2t+1 (token 2 grp + t/2)
+    constexpr int GT = G >= 4 ? 1 : G;   // four groups read theirs per group (below)
+    int Ta[GT], Tb[GT];
+    float F[GT];
 #pragma unroll
-    for (int ks = 0; ks < 8; ks += 2) {
-        mma_16816(c, a0[2 * ks], a1[2 * ks], a0[2 * ks + 1], a1[2 * ks + 1], b[2 * ks], b[2 * ks + 1]);
-        mma_16816(d, a0[2 * ks + 2], a1[2 * ks + 2], a0[2 * ks + 3], a1[2 * ks + 3], b[2 * ks + 2],
-                  b[2 * ks + 3]);
+    for (int grp = 0; grp < GT; ++grp) {
+        const uint32_t tc = 2u * grp + (uint32_t)(t >> 1);
+        uint4 tf = make_uint4(0u, 0u, 0u, 0u);
+        if (tc < Mg) tf = *reinterpret_cast<const uint4*>(xlo + tc * XQD_VAR + XQD_DIGITS * 128);
+        Ta[grp] = (int)(odd ? tf.z : tf.x);
+        Tb[grp] = odd ? 0 : (int)tf.y;
+        F[grp] = __uint_as_float(tf.w);
     }
-    const float s0 = __half2float(__ushort_as_half(sc16[r0]));
-    const float s1 = __half2float(__ushort_as_half(sc16[r1]));
-    const float v0 = s0 * (Fa * (c[0] + d[0]));
-    const float v2 = s1 * (Fa * (c[2] + d[2]));
-    const float v1 = ONE_TOKEN ? 0.f : s0 * (Fb * (c[1] + d[1]));
-    const float v3 = ONE_TOKEN ? 0.f : s1 * (Fb * (c[3] + d[3]));
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {   // acc[rt] without run-time register indexing
-        if (k == rt) {
-            acc[k][0] += v0;
-            acc[k][2] += v2;
-            if (!ONE_TOKEN) { acc[k][1] += v1; acc[k][3] += v3; }
-        }
+    uint32_t bl[8], bh[8];
+    if (G == 1) {
+        load8(bsrc(xlo, 0), bl);
+        if (P1) load8(bsrc(xhi, 0), bh);
     }
-}
-
-template <int B, bool ONE_TOKEN>
-__device__ __forceinline__ void block_accumulate(const uint8_t* stage, const uint32_t (&b)[16], int g,
-                                                 int t, float Fa, float Fb, float (&acc)[4][4]) {
 #pragma unroll 1
-    for (int rt = 0; rt < 4; ++rt) tile_accumulate<B, ONE_TOKEN>(stage, b, rt, g, t, Fa, Fb, acc);
-}
-
-__device__ __forceinline__ void load_bfrag(const uint8_t* src, uint32_t (&b)[16]) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    for (int go = 0; go < (kGroupOuter ? G : 1); ++go) {
+        // the group's digit sums and F, and its accumulators (selected
+        // without run-time register indexing)
+        int Tag = 0, Tbg = 0;
+        float Fg = 0.f;
+        if (kGroupOuter) {
+            const uint32_t tc = 2u * go + (uint32_t)(t >> 1);
+            uint4 tf = make_uint4(0u, 0u, 0u, 0u);
+            if (tc < Mg) tf = *reinterpret_cast<const uint4*>(xlo + tc * XQD_VAR + XQD_DIGITS * 128);
+            Tag = (int)(odd ? tf.z : tf.x);
+            Tbg = odd ? 0 : (int)tf.y;
+            Fg = __uint_as_float(tf.w);
+        }
+        float cur[4];
+        if (kGroupOuter) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint4 v = s4[i];
-        b[4 * i] = v.x; b[4 * i + 1] = v.y; b[4 * i + 2] = v.z; b[4 * i + 3] = v.w;
+            for (int i = 0; i < 4; ++i) {
+                cur[i] = acc[i][0];
+#pragma unroll
+                for (int k = 1; k < G; ++k) cur[i] = (go == k) ? acc[i][k] : cur[i];
+            }
+        }
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt) {
+            const int r0 = 8 * g + 2 * rt;
+            const __half2 sh = bits_h2(*reinterpret_cast<const uint32_t*>(sz + 2 * r0));
+            const __half2 zh = bits_h2(*reinterpret_cast<const uint32_t*>(sz + 128 + 2 * r0));
+            // z is an fp16 integer <= 255: z + 1024 has the bits 0x6400 | z
+            const uint32_t zb = h2_bits(__hadd2(zh, bits_h2(0x64006400u)));
+            const int z0 = (int)(zb & 0x3FFu), z1 = (int)((zb >> 16) & 0x3FFu);
+            const float s_own = __half2float(odd ? __high2half(sh) : __low2half(sh));
+            uint32_t a0[8], a1[8];
+            piece_regs<P0, 0>(lo + r0 * 16 * P0, t, a0);
+            piece_regs<P0, 0>(lo + (r0 + 1) * 16 * P0, t, a1);
+            uint32_t h0[8], h1[8];
+            if (P1) {
+                piece_regs<P1, P0>(hi + r0 * 16 * P1, t, h0);
+                piece_regs<P1, P0>(hi + (r0 + 1) * 16 * P1, t, h1);
+            }
+#pragma unroll
+            for (int gi = 0; gi < (kGroupOuter ? 1 : G); ++gi) {
+                const int grp = kGroupOuter ? 0 : gi;     // register index (group-outer: cur[])
+                const int gsel = kGroupOuter ? go : gi;   // the token group
+                if (G > 1) {
+                    load8(bsrc(xlo, gsel), bl);
+                    if (P1) load8(bsrc(xhi, gsel), bh);
+                }
+                int c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int j = 0; j < 4; j += 2) {
+                    imma_16832(c, a0[2 * j], a1[2 * j], a0[2 * j + 1], a1[2 * j + 1], bl[2 * j], bl[2 * j + 1]);
+                    imma_16832(d, a0[2 * j + 2], a1[2 * j + 2], a0[2 * j + 3], a1[2 * j + 3], bl[2 * j + 2],
+                               bl[2 * j + 3]);
+                }
+                if (P1) {
+#pragma unroll
+                    for (int j = 0; j < 4; j += 2) {
+                        imma_16832(c, h0[2 * j], h1[2 * j], h0[2 * j + 1], h1[2 * j + 1], bh[2 * j],
+                                   bh[2 * j + 1]);
+                        imma_16832(d, h0[2 * j + 2], h1[2 * j + 2], h0[2 * j + 3], h1[2 * j + 3],
+                                   bh[2 * j + 2], bh[2 * j + 3]);
+                    }
+                }
+                // exact int32 parts of rows r0 (c0, c1) and r0 + 1 (c2, c3):
+                // even lanes E_0 + 256 E_1, odd lanes E_2
+                const int ta = kGroupOuter ? Tag : Ta[grp], tb = kGroupOuter ? Tbg : Tb[grp];
+                const int p0 = (c[0] + d[0] - z0 * ta) + 256 * (c[1] + d[1] - z0 * tb);
+                const int p1 = (c[2] + d[2] - z1 * ta) + 256 * (c[3] + d[3] - z1 * tb);
+                // even lane keeps row r0 and gets its E_2; odd lane keeps row r0 + 1
+                const int other = __shfl_xor_sync(0xffffffffu, odd ? p0 : p1, 1);
+                const float lo01 = (float)(odd ? other : p0);
+                const float e2 = (float)(odd ? p1 : other);
+                if (kGroupOuter)
+                    cur[rt] = fmaf(s_own * Fg, fmaf(65536.f, e2, lo01), cur[rt]);
+                else
+                    acc[rt][grp] = fmaf(s_own * F[grp], fmaf(65536.f, e2, lo01), acc[rt][grp]);
+            }
+        }
+        if (kGroupOuter) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int k = 0; k < G; ++k) acc[i][k] = (go == k) ? cur[i] : acc[i][k];
+        }
     }
 }
 
 // Stage layout in the ring (all parts 16-byte multiples):
-//   payload 1024*b | scales 128 | zeros 128 | x' variant of the low piece,
-//   272 bytes per token (fragments, then F)
+//   payload 1024*b | scales 128 | zeros 128 | activation variant of the low
+//   piece, 272 bytes per token | (split widths) the high piece's variant
+__host__ __device__ constexpr bool split_width(int b) { return hi_width(b) != 0; }
 __device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
-    return 1024u * b + 256u + XQD_VAR * Mg;
+    return 1024u * b + 256u + XQD_VAR * Mg * (split_width((int)b) ? 2u : 1u);
 }
 
 // Last arriver of a shared block row: y[m][rows[r]] = sum over the row's nc
@@ -351,13 +382,13 @@ __device__ __noinline__ void finish_shared_row(const float* __restrict__ slots, 
 }
 
 // ---------------------------------------------------------------------------
-// Fused activation record (one token, no prologue kernel): the record that
-// k_xprep_decode would write for block column kb and piece-width variant vv,
-// built by the warp into `rec` (shared memory, XQD_VAR bytes): the slice
-// x[m][col_perm[128kb + c]], c = 0..127, scaled by its power of two 2^e and
-// converted to fp16, paired in the variant's column order, then
-// F = 2^(24 - e) -- the same arithmetic as k_xprep_decode.  cp holds the
-// column indices 128kb + 4 lane .. +3 (after col_perm).
+// Fused activation records (one token, no prologue kernel): the records that
+// k_xprep_decode would write for block column kb, built by the warp in the
+// stage -- the slice x[m][col_perm[128kb + c]], c = 0..127, turned into
+// integers X with its power of two (xqd_integerize), then the digits of the
+// low piece's variant and, for a split width, the high piece's, each
+// followed by the digit sums and F -- the same arithmetic as k_xprep_decode.  cp holds the column indices 128kb + 4 lane .. +3 (after
+// col_perm).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int4 fused_cols(const DecodeParams& p, uint32_t kb, int lane) {
     const int c0 = (int)kb * 128 + 4 * lane;
@@ -365,41 +396,18 @@ __device__ __forceinline__ int4 fused_cols(const DecodeParams& p, uint32_t kb, i
     return __ldg(reinterpret_cast<const int4*>(p.col_perm + c0));
 }
 
-__device__ __forceinline__ void fused_record(const DecodeParams& p, int4 cp, int vv, uint8_t* rec,
-                                             __half* xw, int lane) {
+__device__ __forceinline__ void fused_records(const DecodeParams& p, int4 cp, int b, uint8_t* rec, int lane) {
     const uint16_t* xr = p.x + (size_t)p.m0 * p.K;
     float v[4];
     v[0] = __uint_as_float((uint32_t)xr[cp.x] << 16);
     v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
     v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
     v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
-    float amax = 0.f;
-#pragma unroll
-    for (int e4 = 0; e4 < 4; ++e4) {
-        const float a = fabsf(v[e4]);
-        amax = (a > amax || a != a) ? a : amax;   // NaN-propagating max
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const float o = __shfl_xor_sync(0xffffffffu, amax, off);
-        amax = (o > amax || o != o) ? o : amax;
-    }
-    int e = 0;
-    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -103), 126);
-#pragma unroll
-    for (int e4 = 0; e4 < 4; ++e4) xw[4 * lane + e4] = __float2half_rn(ldexpf(v[e4], e));
-    __syncwarp();
-    // lane -> quad lane tq = lane / 8, pairs 2 (lane % 8), +1
-    const int tq = lane >> 3, pi0 = 2 * (lane & 7);
-    uint32_t o[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        int ca, cb;
-        xqd_pair_cols(vv, pi0 + i, ca, cb);
-        o[i] = h2_bits(__halves2half2(xw[32 * tq + ca], xw[32 * tq + cb]));
-    }
-    *reinterpret_cast<uint2*>(rec + tq * 64 + pi0 * 4) = make_uint2(o[0], o[1]);
-    if (lane == 0) *reinterpret_cast<float*>(rec + 256) = ldexpf(1.f, 24 - e);
+    int X[4], T[3];
+    float F;
+    xqd_integerize(v, X, T, F);
+    xqd_scatter_variant(X, T, F, variant_of(lo_width(b)), rec, lane);
+    if (split_width(b)) xqd_scatter_variant(X, T, F, variant_of(hi_width(b)), rec + XQD_VAR, lane);
     // generic writes into the ring, later overwritten by bulk copies
     fence_proxy_async_smem();
     __syncwarp();
@@ -407,125 +415,94 @@ __device__ __forceinline__ void fused_record(const DecodeParams& p, int4 cp, int
 
 // ---------------------------------------------------------------------------
 // One warp's run u of the layer p (the body of the decode kernels below).
+// G token groups of two: the launch's tokens Mg <= 2G.
 // ---------------------------------------------------------------------------
-template <bool ONE_TOKEN, bool FUSED_X>
+template <int G, bool FUSED_X>
 __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, int u, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const uint32_t KB = (uint32_t)p.KB;
-    const uint32_t lt_mask = (1u << lane) - 1u;
     if (u >= p.n_units) return;
 
-    // ---- the unit descriptor: lane i holds word i ----
+    // ---- the run descriptor: lane i holds word i ----
     const uint32_t dw = __ldg(p.desc + (size_t)u * DESC_WORDS + lane);
     const uint32_t t0 = __shfl_sync(0xffffffffu, dw, DW_T0);
     const uint32_t t1 = __shfl_sync(0xffffffffu, dw, DW_T1);
-    uint32_t sz_base = __shfl_sync(0xffffffffu, dw, DW_SZ);
-    // lanes DW_CODE..DW_CODE+6 keep the running code offset of their width
-    uint32_t code_run = dw;
-
+    const uint32_t s0 = __shfl_sync(0xffffffffu, dw, DW_S0);
+    const uint32_t ns = __shfl_sync(0xffffffffu, dw, DW_NS);
 
     const uint32_t Mg = (uint32_t)p.Mg;
     // xq offsets fit 32 bits: KB * M * XQD_REC < 2^32 (the host checks it)
     const uint32_t rec_bytes = (uint32_t)p.M_total * XQD_REC;
     const uint32_t var_bytes = (uint32_t)p.M_total * XQD_VAR;
     const uint32_t x_tok_off = (uint32_t)p.m0 * XQD_VAR;
-    const uint32_t x_bytes = XQD_VAR * Mg;
+    const uint32_t x_bytes = XQD_VAR * Mg;     // one variant of the launch's tokens
 
-    // ---- chunk state: lane l describes block t0 + 32*chunk + l ----
+    // ---- stage descriptors of the current chunk: lane l holds stage 32 chunk + l ----
     uint32_t chunk = 0;
-    uint32_t c_bits = 0, c_code = 0, c_sz = 0, c_x = 0;
-    uint32_t pending = 0;            // non-zero blocks of the chunk not yet issued
-    bool scan_done = false;
-    uint32_t bits_pref = 0;          // prefetched widths of the next chunk (beyond the inline 64)
-
-    bool aborted = false;            // a bounded wait ran out: stop computing
+    uint4 cs = make_uint4(0u, 0u, 0u, 0u);
     auto load_chunk = [&]() {
         const uint32_t j = 32u * chunk + (uint32_t)lane;
-        const bool in = t0 + j < t1;
-        // widths of the first 64 blocks are inline in the descriptor
-        const uint32_t jw = min(j, (uint32_t)DESC_INLINE_BITS - 1u);
-        const uint32_t word = __shfl_sync(0xffffffffu, dw, DW_BITS + (int)(jw >> 2));
-        uint32_t b = (j < (uint32_t)DESC_INLINE_BITS) ? (word >> (8 * (j & 3))) & 0xFFu : bits_pref;
-        b = in ? b : 0u;
-        // prefetch the next chunk's widths when they are not inline
-        const uint32_t jn = j + 32u;
-        if (jn >= (uint32_t)DESC_INLINE_BITS && t0 + jn < t1) bits_pref = __ldg(p.bits8 + t0 + jn);
-        c_bits = b;
-        // this block's activation variant for the launch's tokens, as a byte
-        // offset into xq (one division per chunk instead of one per stage)
-        c_x = ((t0 + j) % KB) * rec_bytes + (uint32_t)variant_of(lo_width(b == 0 ? 1 : (int)b)) * var_bytes +
-              x_tok_off;
-        // rank among the chunk's blocks of the same width -> code offset
-        const uint32_t same = __match_any_sync(0xffffffffu, b);
-        const uint32_t rank = __popc(same & lt_mask);
-        const uint32_t base = __shfl_sync(0xffffffffu, code_run, DW_CODE + width_index(b == 0 ? 1 : (int)b));
-        c_code = base + rank * 1024u * b;
-        const uint32_t nz = __ballot_sync(0xffffffffu, b != 0u);
-        c_sz = sz_base + 64u * __popc(nz & lt_mask);
-        sz_base += 64u * __popc(nz);
-        pending = nz;
+        if (j < ns) cs = __ldg(p.stages + s0 + j);
     };
-    // advance the running code offsets past the chunk (lane DW_CODE + i owns width i)
-    auto advance_codes = [&]() {
-        uint32_t add = 0;
-#pragma unroll
-        for (int i = 0; i < 7; ++i) {
-            const uint32_t wb = (i == 6) ? 8u : (uint32_t)(i + 1);
-            const uint32_t cnt = __popc(__ballot_sync(0xffffffffu, c_bits == wb));
-            if (lane == DW_CODE + i) add = cnt * 1024u * wb;
-        }
-        code_run += add;
-    };
-
     load_chunk();
-    advance_codes();
+    uint32_t next = 0;               // stages issued
+
+    bool aborted = false;            // a bounded wait ran out: stop computing
+    // variant of piece width p's activation record: 1, 2, 4, 8 -> 0, 1, 2, 3;
+    // the low piece of width b is variant (0x302221100 >> 4b) & 15
+    auto var_lo = [](uint32_t b) -> uint32_t { return (uint32_t)(0x302221100ull >> (4 * b)) & 15u; };
+    auto var_hi = [](uint32_t b) -> uint32_t { return (uint32_t)(0x001010000ull >> (4 * b)) & 15u; };
+    auto issue_x = [&](uint8_t* dst, uint32_t b, uint32_t xo, uint64_t* bar) {
+        bulk_g2s(dst, p.xq + xo, x_bytes, bar);
+        // the high piece is narrower: its variant comes first in the record
+        if (split_width((int)b))
+            bulk_g2s(dst + x_bytes, p.xq + (xo - (var_lo(b) - var_hi(b)) * var_bytes), x_bytes, bar);
+    };
 
     // ---- stage queue: entry k lives in lane k % DEC_SLOTS ----
     uint32_t q_head = 0, q_tail = 0;     // consumed / issued stages
     uint32_t r_head = 0, r_tail = 0;     // ring bytes issued / freed (monotone)
     uint32_t r_pos = 0;                  // physical ring offset of r_head
-    uint32_t qe_t = 0, qe_bits = 0, qe_off = 0, qe_end = 0, qe_x = 0;
+    uint32_t qe_nb = 0, qe_bits = 0, qe_off = 0, qe_end = 0, qe_x = 0, qe_kb = 0;
     bool xq_ready = false;               // x' is written by the prologue kernel
     auto issue_more = [&]() {
-        while (q_tail - q_head < (uint32_t)DEC_SLOTS && !scan_done) {
-            if (aborted) { scan_done = true; break; }
-            if (pending == 0u) {
-                if (t0 + 32u * (chunk + 1) >= t1) { scan_done = true; break; }
-                ++chunk;
-                load_chunk();
-                advance_codes();
-                continue;
-            }
+        while (q_tail - q_head < (uint32_t)DEC_SLOTS && next < ns && !aborted) {
+            const int l = (int)(next & 31u);
+            const uint32_t coff = __shfl_sync(0xffffffffu, cs.x, l);
+            const uint32_t szo = __shfl_sync(0xffffffffu, cs.y, l);
+            const uint32_t kbb = __shfl_sync(0xffffffffu, cs.z, l);
+            const uint32_t nbs = __shfl_sync(0xffffffffu, cs.w, l);
+            const uint32_t b = kbb >> 16;
+            const uint32_t xo = (kbb & 0xFFFFu) * rec_bytes + var_lo(b) * var_bytes + x_tok_off;
+            const uint32_t xb = split_width((int)b) ? 2u * x_bytes : x_bytes;
+            const uint32_t size = 1024u * b + 256u + xb;   // stage_bytes(b, Mg)
             if (q_head == q_tail) { r_head = 0; r_tail = 0; r_pos = 0; }   // empty ring: restart at 0
-            const int l = __ffs(pending) - 1;
-            const uint32_t b = __shfl_sync(0xffffffffu, c_bits, l);
-            const uint32_t coff = __shfl_sync(0xffffffffu, c_code, l);
-            const uint32_t szo = __shfl_sync(0xffffffffu, c_sz, l);
-            const uint32_t xo = __shfl_sync(0xffffffffu, c_x, l);
-            const uint32_t size = 1024u * b + 256u + x_bytes;   // stage_bytes(b, Mg)
             // a stage never wraps: when the ring's tail end is too short, skip to 0
             const bool skip = r_pos + size > (uint32_t)DEC_RING;
             const uint32_t start = skip ? r_head + ((uint32_t)DEC_RING - r_pos) : r_head;
             if (start + size - r_tail > (uint32_t)DEC_RING) break;   // ring full: compute first
-            const uint32_t tt = t0 + 32u * chunk + (uint32_t)l;
             const uint32_t slot = q_tail % DEC_SLOTS;
             const uint32_t off = skip ? 0u : r_pos;
             if (lane == 0) {
-                fence_proxy_async_smem();
+                // the fused path writes activation records into the ring
+                if (FUSED_X) fence_proxy_async_smem();
                 uint64_t* bar = &W.full[slot];
-                // the fused path builds the activation record itself
-                mbar_arrive_expect_tx(bar, FUSED_X ? size - x_bytes : size);
+                mbar_arrive_expect_tx(bar, FUSED_X ? size - xb : size);
                 uint8_t* dst = W.ring + off;
                 bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
                 bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
                 bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
-                if (!FUSED_X && xq_ready) bulk_g2s(dst + 1024u * b + 256u, p.xq + xo, x_bytes, bar);
+                if (!FUSED_X && xq_ready) issue_x(dst + 1024u * b + 256u, b, xo, bar);
             }
-            if (lane == (int)slot) { qe_t = tt; qe_bits = b; qe_off = off; qe_end = start + size; qe_x = xo; }
+            if (lane == (int)slot) {
+                qe_nb = nbs; qe_bits = b; qe_off = off; qe_end = start + size; qe_x = xo;
+                if (FUSED_X) qe_kb = kbb & 0xFFFFu;
+            }
             r_head = start + size;
             r_pos = off + size;
             ++q_tail;
-            pending &= pending - 1u;
+            ++next;
+            if ((next & 31u) == 0u) { ++chunk; load_chunk(); }
         }
     };
 
@@ -537,7 +514,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
     int4 cp_pref = make_int4(0, 0, 0, 0);
     uint32_t cp_kb = 0xFFFFFFFFu;
     if (FUSED_X && q_head != q_tail) {
-        cp_kb = __shfl_sync(0xffffffffu, qe_t, q_head % DEC_SLOTS) % KB;
+        cp_kb = __shfl_sync(0xffffffffu, cs.z, 0) & 0xFFFFu;   // the run's first non-zero block
         cp_pref = fused_cols(p, cp_kb, lane);
     }
     pdl_wait();
@@ -548,32 +525,33 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
             const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
-            if (lane == 0) bulk_g2s(W.ring + ko + 1024u * kbits + 256u, p.xq + kx, x_bytes, &W.full[slot]);
+            if (lane == 0) issue_x(W.ring + ko + 1024u * kbits + 256u, kbits, kx, &W.full[slot]);
         }
     }
 
     const uint32_t nb_first = t0 / KB, nb_last = (t1 - 1) / KB;
     for (uint32_t nb = nb_first; nb <= nb_last; ++nb) {
-        const uint32_t row_end = min(t1, (nb + 1) * KB);
-        // output rows of this lane: 16rt+g (+8); their permuted indices, early
-        int rp[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int i = (int)nb * 64 + 8 * q + g;   // q = 2rt + h -> row 16rt + 8h + g
-            rp[q] = p.row_perm ? __ldg(p.row_perm + i) : i;
+        // output indices of the block row's 64 rows, kept in shared memory
+        // (fetched early; read back when the row is written)
+        __syncwarp();
+        if (lane < 16) {
+            const int i0 = (int)nb * 64 + 4 * lane;
+            const int4 r4 = p.row_perm ? __ldg(reinterpret_cast<const int4*>(p.row_perm + i0))
+                                       : make_int4(i0, i0 + 1, i0 + 2, i0 + 3);
+            *reinterpret_cast<int4*>(&W.rows[4 * lane]) = r4;
         }
-        float acc[4][4];
+        float acc[4][G];      // rows 8g + 2i + (t & 1), token 2 grp + t / 2
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+            for (int c = 0; c < G; ++c) acc[i][c] = 0.f;
 
         while (true) {
             issue_more();
             if (q_head == q_tail) break;    // nothing left for this warp at all
             const uint32_t slot = q_head % DEC_SLOTS;
-            const uint32_t ft = __shfl_sync(0xffffffffu, qe_t, slot);
-            if (ft >= row_end) break;       // the next block is in a later row
+            const uint32_t fnb = __shfl_sync(0xffffffffu, qe_nb, slot);
+            if (fnb != nb) break;           // the next block is in a later row
             const uint32_t fb = __shfl_sync(0xffffffffu, qe_bits, slot);
             const uint32_t foff = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t fend = __shfl_sync(0xffffffffu, qe_end, slot);
@@ -586,28 +564,22 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             }
             if (!aborted) {
                 const uint8_t* stage = W.ring + foff;
-                const uint8_t* xs = stage + 1024u * fb + 256u;
+                uint8_t* xs = W.ring + foff + 1024u * fb + 256u;
                 if (FUSED_X) {
-                    const uint32_t kb = ft % KB;
+                    const uint32_t kb = __shfl_sync(0xffffffffu, qe_kb, slot);
                     const int4 cp = (kb == cp_kb) ? cp_pref : fused_cols(p, kb, lane);
-                    fused_record(p, cp, variant_of(lo_width((int)fb)), W.ring + foff + 1024u * fb + 256u,
-                                 W.xw, lane);
+                    fused_records(p, cp, (int)fb, xs, lane);
                 }
-                // this lane's B fragments: token g, quad lane t; zeros beyond Mg
-                uint32_t bf[16];
-                load_bfrag((uint32_t)g < Mg ? xs + g * XQD_VAR + t * 64
-                                            : reinterpret_cast<const uint8_t*>(W.zero16), bf);
-                const float Fa = (2u * t < Mg) ? *reinterpret_cast<const float*>(xs + (2 * t) * XQD_VAR + 256) : 0.f;
-                const float Fb = (!ONE_TOKEN && 2u * t + 1u < Mg)
-                                     ? *reinterpret_cast<const float*>(xs + (2 * t + 1) * XQD_VAR + 256) : 0.f;
+                const uint8_t* xh = xs + x_bytes;
+                const uint8_t* z32 = reinterpret_cast<const uint8_t*>(W.zero32);
                 switch (fb) {
-                    case 1: block_accumulate<1, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
-                    case 2: block_accumulate<2, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
-                    case 3: block_accumulate<3, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
-                    case 4: block_accumulate<4, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
-                    case 5: block_accumulate<5, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
-                    case 6: block_accumulate<6, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
-                    default: block_accumulate<8, ONE_TOKEN>(stage, bf, g, t, Fa, Fb, acc); break;
+                    case 1: block_accumulate<1, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
+                    case 2: block_accumulate<2, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
+                    case 3: block_accumulate<3, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
+                    case 4: block_accumulate<4, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
+                    case 5: block_accumulate<5, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
+                    case 6: block_accumulate<6, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
+                    default: block_accumulate<8, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
                 }
             }
             __syncwarp();
@@ -626,31 +598,32 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             nc = __shfl_sync(0xffffffffu, dw, DW_B_NC);
             idx = __shfl_sync(0xffffffffu, dw, DW_B_IDX);
         }
-        // tokens 2t, 2t+1 of rows 16rt+g, 16rt+g+8
-        const int tok_a = 2 * t, tok_b = 2 * t + 1;
-        const bool wa = (uint32_t)tok_a < Mg, wb = !ONE_TOKEN && (uint32_t)tok_b < Mg;
+        // this lane's values: rows 8g + 2i + (t & 1) of token 2 grp + t / 2
+        __syncwarp();
+        const int row0 = 8 * g + (t & 1);
         if (nc == 1u) {
 #pragma unroll
-            for (int rt = 0; rt < 4; ++rt)
+            for (int grp = 0; grp < G; ++grp) {
+                const uint32_t tok = 2u * grp + (uint32_t)(t >> 1);
+                if (tok < Mg) {
+                    float* yr = p.y + (size_t)(p.m0 + tok) * p.N;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = rp[2 * rt + h];
-                    if (wa) p.y[(size_t)(p.m0 + tok_a) * p.N + n] = acc[rt][2 * h];
-                    if (wb) p.y[(size_t)(p.m0 + tok_b) * p.N + n] = acc[rt][2 * h + 1];
+                    for (int i = 0; i < 4; ++i) yr[W.rows[row0 + 2 * i]] = acc[i][grp];
                 }
+            }
             continue;
         }
         // shared row: deposit this run's partial sums, then count the arrival
         {
             float* part = p.partial + (size_t)(slot_base + idx) * Mg * 64;
 #pragma unroll
-            for (int rt = 0; rt < 4; ++rt)
+            for (int grp = 0; grp < G; ++grp) {
+                const uint32_t tok = 2u * grp + (uint32_t)(t >> 1);
+                if (tok < Mg) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int r = 16 * rt + 8 * h + g;
-                    if (wa) part[tok_a * 64 + r] = acc[rt][2 * h];
-                    if (wb) part[tok_b * 64 + r] = acc[rt][2 * h + 1];
+                    for (int i = 0; i < 4; ++i) part[tok * 64 + row0 + 2 * i] = acc[i][grp];
                 }
+            }
         }
         // __syncwarp orders every lane's partial before lane 0's release; the
         // acquire side is lane 0's atomic + __syncwarp, then L2 (.cg) loads
@@ -660,11 +633,6 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
         last = __shfl_sync(0xffffffffu, last, 0);
         __syncwarp();
         if (!last) continue;
-        if (t == 0) {   // the row's output indices, for the lanes that write y below
-#pragma unroll
-            for (int q = 0; q < 8; ++q) W.rows[8 * q + g] = rp[q];
-        }
-        __syncwarp();
         finish_shared_row(p.partial + (size_t)slot_base * Mg * 64, Mg, nc, p.y + (size_t)p.m0 * p.N,
                           p.N, W.rows, lane);
         if (lane == 0) p.counters[nb] = 0u;   // ready for the next launch
@@ -673,11 +641,10 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
 
 
 // ---------------------------------------------------------------------------
-// The kernels.  ONE_TOKEN: the launch has Mg == 1 (only C-fragment column 0
-// carries data, so the per-block epilogue handles half the elements).
-// FUSED_X (with ONE_TOKEN): no prologue kernel; each block's activation
-// record is built by the warp from x (fused_record).  Every warp works
-// alone (no CTA-wide barrier): warp u of the grid takes run u.
+// The kernels.  G: token groups of four (Mg <= 4G).  FUSED_X (one token): no
+// prologue kernel; each block's activation records are built by the warp
+// from x (fused_records).  Every warp works alone (no CTA-wide barrier): warp
+// u of the grid takes run u.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ DecWarp& decode_prologue(uint8_t* smem_raw, int warp, int lane) {
     DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
@@ -689,19 +656,24 @@ __device__ __forceinline__ DecWarp& decode_prologue(uint8_t* smem_raw, int warp,
         for (int s = 0; s < DEC_SLOTS; ++s) mbar_init(&W.full[s], 1);
         fence_mbar_init();
     }
-    if (lane < 4) W.zero16[lane] = make_uint4(0u, 0u, 0u, 0u);
+    if (lane < 2) W.zero32[lane] = make_uint4(0u, 0u, 0u, 0u);
     __syncwarp();
     return W;
 }
 
-template <bool ONE_TOKEN, bool FUSED_X = false>
-// At most 112 registers: four CTAs then leave room in the register file for
-// the next launch's activation-prologue CTAs to become resident early.
-__global__ void __maxnreg__(DEC_MAX_REGS) k_decode(DecodeParams p) {
+// Registers: at most 112 for one token group (four CTAs per SM then leave
+// room in the register file for the next launch's prologue CTAs to become
+// resident early); more token groups hold more accumulators and fragments
+// (three CTAs per SM).
+template <int G>
+struct DecRegs { static constexpr int value = G == 1 ? DEC_MAX_REGS : 168; };
+
+template <int G, bool FUSED_X = false>
+__global__ void __maxnreg__(DecRegs<G>::value) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     DecWarp& W = decode_prologue(smem_raw, warp, lane);
-    decode_warp<ONE_TOKEN, FUSED_X>(p, W, (int)blockIdx.x * DEC_WARPS + warp, lane);
+    decode_warp<G, FUSED_X>(p, W, (int)blockIdx.x * DEC_WARPS + warp, lane);
 }
 
 // Several layers that share x in one launch (one token, fused activation
@@ -721,7 +693,7 @@ __global__ void __maxnreg__(DEC_MAX_REGS) k_decode_group(const __grid_constant__
     if (v >= gp.unit_begin[gp.n]) return;
     int l = 0;
     while (l + 1 < gp.n && v >= gp.unit_begin[l + 1]) ++l;
-    decode_warp<true, true>(gp.layer[l], W, v - gp.unit_begin[l], lane);
+    decode_warp<1, true>(gp.layer[l], W, v - gp.unit_begin[l], lane);
 }
 
 }  // namespace mpq

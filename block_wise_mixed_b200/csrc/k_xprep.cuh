@@ -8,15 +8,9 @@
 // (e_m = 14 - floor(log2(amax_m)), so amax*2^e lies in [2^14, 2^15)); the
 // GEMM epilogues multiply by tok_scale[m] = 2^-e_m, which is exact.
 //
-// Layouts written:
-//   XP_DECODE : [KB][M][4][16] half2 -- for block column kb, token m and quad
-//               lane t, register r = 4i+j holds the columns (32t+8i+j,
-//               32t+8i+j+4) of that block column: exactly the B fragment of
-//               mma.m16n8k16 that the decode kernel pairs with its code
-//               extraction order.
-//   XP_PREFILL: [M][K] half, K contiguous, each 128-column group permuted so
-//               that position 2*(4i+j)+h holds column 8i+j+4h -- the order in
-//               which the tensor-core kernel's dequantization emits weights.
+// Layout written (XP_PREFILL): [M][K] half, K contiguous, each 128-column
+// group permuted so that position 2*(4i+j)+h holds column 8i+j+4h -- the
+// order in which the tensor-core kernel's dequantization emits weights.
 // Block 0 also clears the decode kernel's per-block-row counters (when given).
 //
 // k_xprep_decode (below) is the small-batch variant; its layout is described
@@ -90,18 +84,7 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
         int c = p.col_perm ? p.col_perm[j] : j;
         return ldexpf(__uint_as_float(((uint32_t)xr[c]) << 16), e);
     };
-    if (LAYOUT == XP_DECODE) {
-        const int KB = K / 128;
-        __half2* out = reinterpret_cast<__half2*>(p.xq);
-        for (int idx = tid; idx < K / 2; idx += XPREP_THREADS) {
-            const int kb = idx >> 6, rem = idx & 63;
-            const int t = rem >> 4, r = rem & 15, i = r >> 2, j = r & 3;
-            const int col = kb * 128 + 32 * t + 8 * i + j;
-            __half2 v = __halves2half2(__float2half_rn(load(col)), __float2half_rn(load(col + 4)));
-            out[((size_t)kb * p.M + m) * 64 + rem] = v;
-        }
-        (void)KB;
-    } else {
+    {
         __half2* out = reinterpret_cast<__half2*>(p.xq + (size_t)m * K);
         for (int c2 = tid; c2 < K / 2; c2 += XPREP_THREADS) {
             const int kb = c2 >> 6, r = c2 & 63, i = r >> 2, j = r & 3;
@@ -114,52 +97,144 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
 // ---------------------------------------------------------------------------
 // Small-batch activation records (k_xprep_decode).
 //
-// The decode kernel turns a pair of packed codes into the fp16 pair
-// ((q_a - z) * 2^-24, (q_b - z) * 2^-24) -- exact subnormals -- with one AND
-// (or byte permute) and one HFMA2 per pair.  Which two columns share a pair
-// follows from where a p-bit piece puts its codes in a 32-bit word (the two
-// 16-bit halves), so each piece width p = 1, 2, 4, 8 pairs the columns in its
-// own order, and the activation slice is stored once per order ("variant").
-// For quad lane t of the mma, pair index pi (0..15) of a row's 32 columns
-// 32t..32t+31 holds the columns (colA, colB):
-//   p = 1: cols (s + 8*(pi/8), s + 8*(pi/8) + 16),  s = pi % 8
-//   p = 2: cols (16i + 4h + s, 16i + 4h + s + 8),   i = pi/8, h = (pi/4)%2, s = pi%4
-//   p = 4: cols (8i + r, 8i + r + 4),               i = pi/4, r = pi % 4
-//   p = 8: cols (4i + r, 4i + r + 2),               i = pi/2, r = pi % 2
-// and register pi of the mma B fragment is (x'[colA], x'[colB]).
+// The decode kernel multiplies packed codes by activations on the integer
+// tensor cores (mma.m16n8k32, u8 codes x s8 activations, s32 accumulation),
+// so every product and every sum is exact.  Each 128-column slice (block
+// column kb) of token m is turned into integers by its own power of two:
+//   e = 22 - floor(log2 amax)  (one less if amax * 2^e would exceed XQD_XMAX),
+//   X_c = rne(x'_c * 2^e),  |X_c| <= XQD_XMAX < 2^23,
+// which is exact for every element within a factor 2^15 of the slice maximum
+// (bf16 carries 8 significant bits) and otherwise off by at most half a unit
+// (2^-23 of the slice maximum).  X = d0 + 256 d1 + 65536 d2 with every digit
+// in [-128, 127]: three s8 "digits", three columns of the mma's B operand.
+// With T_d = sum_c d_d(X_c) (exact), the decode kernel forms per output row
+//   E_d = sum_c (q_c - z) d_d(X_c) = C_d - z T_d                (int32, exact)
+//   V   = E_0 + 256 E_1 + 65536 E_2 = sum_c (q_c - z) X_c
+// and adds s * F * V with F = 2^-e (a non-finite slice gives F = NaN, so
+// non-finite x gives non-finite y).
 //
-// Each 128-column slice (block column kb) of token m is scaled by its own
-// power of two 2^e (amax * 2^e in [2^14, 2^15), e >= -103), so that bf16
-// values are exact in fp16.  The tensor cores then accumulate
-// c_r = 2^-24 * sum_j (q_j - z_r) x'_j, and the block adds s_r * F * c_r to
-// output row r, with F = 2^(24 - e).
+// The kernel unpacks four codes of one 32-bit code word into the four bytes
+// of a register with one AND (a "plane" of the word), so the column order
+// of the A operand depends on the piece width p that the codes come from.
+// For k-tile j (32 columns of the A operand), register half hf (mma
+// registers a0/a1 vs a2/a3), quad lane t and byte b, the operand column
+// kappa = 32j + 16hf + 4t + b holds the code of slice column
+//   p = 1:  32t + 8b + 2j + hf
+//   p = 2:  32t + 16(j/2) + 4b + 2(j%2) + hf
+//   p = 4:  32t + 8j + 2b + hf
+//   p = 8:  32t + 8j + 4hf + b
+// (xqd_col below), and each width has its own copy ("variant") of the slice.
 //
 // Record of block column kb (XQD_REC * M bytes, 16-byte aligned): for each
-// variant v = 0..3 (p = 1, 2, 4, 8) and token m, XQD_VAR = 272 bytes:
-//   [t = 0..3][pi = 0..15] half2 (256 B), then F as float4 (F, 0, 0, 0)
-// so one variant of a token group is one contiguous run of 272*Mg bytes.
+// variant v = 0..3 (p = 1, 2, 4, 8) and token m, XQD_VAR = 400 bytes:
+//   [d = 0..2][t = 0..3][j = 0..3][hf = 0, 1][b = 0..3] s8: digit d of X at
+//   column kappa -- for quad lane t and mma column d, the 32 bytes are its
+//   B-fragment registers of the four k-tiles in order;
+//   then T_0, T_1, T_2 (int32) and F (float).
+// so one variant of a token group is one contiguous run of 400*Mg bytes.
 // Block 0 also clears the decode kernel's per-block-row counters.
 // ---------------------------------------------------------------------------
-constexpr int XQD_VAR = 272;                 // one variant of one token: fragments + F
+constexpr int XQD_DIGITS = 3;
+constexpr int XQD_VAR = XQD_DIGITS * 128 + 16;   // one variant of one token: digits, T_d, F
 constexpr int XQD_REC = 4 * XQD_VAR;
+constexpr float XQD_XMAX = 8355711.f;            // 127 * (1 + 256 + 65536): three s8 digits
 
-__device__ __forceinline__ void xqd_pair_cols(int v, int pi, int& ca, int& cb) {
-    if (v == 0) {
-        ca = (pi & 7) + 8 * (pi >> 3); cb = ca + 16;
-    } else if (v == 1) {
-        ca = 16 * (pi >> 3) + 4 * ((pi >> 2) & 1) + (pi & 3); cb = ca + 8;
-    } else if (v == 2) {
-        ca = 8 * (pi >> 2) + (pi & 3); cb = ca + 4;
-    } else {
-        ca = 4 * (pi >> 1) + (pi & 1); cb = ca + 2;
+__host__ __device__ __forceinline__ int xqd_col(int v, int kappa) {
+    const int j = kappa >> 5, hf = (kappa >> 4) & 1, t = (kappa >> 2) & 3, b = kappa & 3;
+    if (v == 0) return 32 * t + 8 * b + 2 * j + hf;
+    if (v == 1) return 32 * t + 16 * (j >> 1) + 4 * b + 2 * (j & 1) + hf;
+    if (v == 2) return 32 * t + 8 * j + 2 * b + hf;
+    return 32 * t + 8 * j + 4 * hf + b;
+}
+
+// Balanced base-256 digit d of X (|X| <= XQD_XMAX).
+__device__ __forceinline__ int xqd_digit(int X, int d) {
+    const int d0 = ((X + 128) & 255) - 128;
+    if (d == 0) return d0;
+    const int X1 = (X - d0) >> 8;
+    const int d1 = ((X1 + 128) & 255) - 128;
+    if (d == 1) return d1;
+    return (X1 - d1) >> 8;
+}
+
+// Byte position of slice column c within a digit row of variant v: the
+// inverse of xqd_col (kappa = 32j + 16hf + 4t + b is stored at 32t + 8j +
+// 4hf + b).
+__host__ __device__ __forceinline__ int xqd_pos(int v, int c) {
+    const int t = c >> 5, r = c & 31;
+    int j, hf, b;
+    if (v == 0) { b = r >> 3; j = (r & 7) >> 1; hf = r & 1; }
+    else if (v == 1) { j = 2 * (r >> 4) + ((r & 3) >> 1); b = (r & 15) >> 2; hf = r & 1; }
+    else if (v == 2) { j = r >> 3; b = (r & 7) >> 1; hf = r & 1; }
+    else { j = r >> 3; hf = (r & 7) >> 2; b = r & 3; }
+    return 32 * t + 8 * j + 4 * hf + b;
+}
+
+// Slice exponent e from the slice's largest magnitude (NaN-propagating max).
+__device__ __forceinline__ int xqd_exponent(float amax) {
+    int e = 0;
+    if (amax > 0.f && isfinite(amax)) {
+        e = 22 - ilogbf(amax);
+        if (ldexpf(amax, e) > XQD_XMAX) e -= 1;
+        e = min(e, 126);
     }
+    return e;
+}
+
+// The slice's integers: the warp's lane holds slice columns 4 lane .. +3
+// (values v[]); X[] receives their integers and T[0..2] the digit sums of
+// the whole slice (every lane); F is 2^-e, or NaN for a non-finite slice.
+__device__ __forceinline__ void xqd_integerize(const float (&v)[4], int (&X)[4], int (&T)[3], float& F) {
+    float amax = 0.f;
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+        const float a = fabsf(v[e4]);
+        amax = (a > amax || a != a) ? a : amax;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, amax, off);
+        amax = (o > amax || o != o) ? o : amax;
+    }
+    const int e = xqd_exponent(amax);
+    T[0] = T[1] = T[2] = 0;
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+        const float sv = ldexpf(v[e4], e);
+        X[e4] = isfinite(sv) ? __float2int_rn(sv) : 0;
+#pragma unroll
+        for (int d = 0; d < 3; ++d) T[d] += xqd_digit(X[e4], d);
+    }
+#pragma unroll
+    for (int d = 0; d < 3; ++d)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) T[d] += __shfl_xor_sync(0xffffffffu, T[d], off);
+    F = isfinite(amax) ? ldexpf(1.f, -e) : __int_as_float(0x7fc00000);
+}
+
+// One variant's record into rec (shared memory, XQD_VAR bytes): each lane
+// stores the three digits of its four columns at their positions, then lane
+// 0 the digit sums and F.
+__device__ __forceinline__ void xqd_scatter_variant(const int (&X)[4], const int (&T)[3], float F, int vv,
+                                                    uint8_t* rec, int lane) {
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+        const int pos = xqd_pos(vv, 4 * lane + e4);
+#pragma unroll
+        for (int d = 0; d < 3; ++d) rec[d * 128 + pos] = (uint8_t)xqd_digit(X[e4], d);
+    }
+    if (lane == 0)
+        *reinterpret_cast<uint4*>(rec + XQD_DIGITS * 128) =
+            make_uint4((uint32_t)T[0], (uint32_t)T[1], (uint32_t)T[2], __float_as_uint(F));
 }
 
 constexpr int XPREP_DEC_WARPS = XPREP_THREADS / 32;
 
-__global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
+__global__ void __launch_bounds__(XPREP_THREADS, 8) k_xprep_decode(XprepParams p) {
     pdl_launch_dependents();
-    __shared__ float xs[XPREP_DEC_WARPS][64];   // 128 fp16 per warp
+    // one variant at a time per warp (small, so that the CTAs fit beside the
+    // decode kernel's on an SM)
+    __shared__ __align__(16) uint8_t recs[XPREP_DEC_WARPS][XQD_VAR];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int KB = p.K / 128;
     const int item = blockIdx.x * XPREP_DEC_WARPS + warp;   // = kb * M + m
@@ -182,41 +257,21 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep_decode(XprepParams p) {
     v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
     v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
     v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
-    float amax = 0.f;
-#pragma unroll
-    for (int e4 = 0; e4 < 4; ++e4) {
-        const float a = fabsf(v[e4]);
-        amax = (a > amax || a != a) ? a : amax;   // NaN-propagating max
+    int X[4], T[3];
+    float F;
+    xqd_integerize(v, X, T, F);
+    uint8_t* rs = recs[warp];
+    // variant vv of token m of block column kb
+    uint8_t* rec = reinterpret_cast<uint8_t*>(p.xq) + (size_t)kb * p.M * XQD_REC + (size_t)m * XQD_VAR;
+#pragma unroll 1
+    for (int vv = 0; vv < 4; ++vv) {
+        xqd_scatter_variant(X, T, F, vv, rs, lane);
+        __syncwarp();
+        if (lane < XQD_VAR / 16)
+            reinterpret_cast<uint4*>(rec + (size_t)vv * p.M * XQD_VAR)[lane] =
+                reinterpret_cast<const uint4*>(rs)[lane];
+        __syncwarp();
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const float o = __shfl_xor_sync(0xffffffffu, amax, off);
-        amax = (o > amax || o != o) ? o : amax;
-    }
-    int e = 0;
-    if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -103), 126);
-    // x' = fp16(x * 2^e) (exact for bf16 inputs in range)
-    __half* xw = reinterpret_cast<__half*>(xs[warp]);
-#pragma unroll
-    for (int e4 = 0; e4 < 4; ++e4) xw[4 * lane + e4] = __float2half_rn(ldexpf(v[e4], e));
-    __syncwarp();
-    // lane -> variant vv = lane / 8, quad lane tq = (lane / 2) % 4, pairs 8*(lane % 2) .. +7
-    const int vv = lane >> 3, tq = (lane >> 1) & 3, pi0 = 8 * (lane & 1);
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int ca, cb;
-        xqd_pair_cols(vv, pi0 + i, ca, cb);
-        o[i] = h2_bits(__halves2half2(xw[32 * tq + ca], xw[32 * tq + cb]));
-    }
-    uint8_t* rec = reinterpret_cast<uint8_t*>(p.xq) + (size_t)kb * p.M * XQD_REC;
-    uint4* dst = reinterpret_cast<uint4*>(rec + (size_t)vv * p.M * XQD_VAR + (size_t)m * XQD_VAR +
-                                          tq * 64 + pi0 * 4);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-    if ((lane & 7) == 0)   // one lane per variant writes F after the fragments
-        *reinterpret_cast<float4*>(rec + (size_t)vv * p.M * XQD_VAR + (size_t)m * XQD_VAR + 256) =
-            make_float4(ldexpf(1.f, 24 - e), 0.f, 0.f, 0.f);
 }
 
 }  // namespace mpq

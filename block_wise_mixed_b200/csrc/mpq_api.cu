@@ -41,13 +41,14 @@ inline uint64_t block_cost(int b) {
     return b == 0 ? 32u : 1024u * (uint64_t)b + 256u + 272u + work[b];
 }
 
-inline uint64_t sched_words_of(int64_t n_units, int64_t T) {
-    return (uint64_t)n_units * DESC_WORDS + (uint64_t)(T + 3) / 4;
+inline uint64_t sched_words_of(int64_t n_units, uint64_t n_stages) {
+    return (uint64_t)n_units * DESC_WORDS + (uint64_t)STAGE_WORDS * n_stages;
 }
 
 // Layout of the plan for (N, K, bits) -- the same arithmetic as mpq_plan.
-// sched (optional) receives the decode schedule: n_units descriptors of
-// DESC_WORDS words (see k_decode.cuh), then one byte per block (its width).
+// sched (optional) receives the decode schedule: n_units run descriptors of
+// DESC_WORDS words (see k_decode.cuh), then one STAGE_WORDS-word stage
+// descriptor per non-zero block, in block order.
 mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
                      std::vector<mpq_block>* table, std::vector<uint32_t>* sched) {
     if (N <= 0 || K <= 0 || N % 64 != 0 || K % 128 != 0) return MPQ_ERR_SHAPE;
@@ -104,8 +105,8 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
     bounds.push_back((uint32_t)T);
     const int64_t units = (int64_t)bounds.size() - 1;
     L->n_units = (int32_t)units;
-    if (sched_words_of(units, T) >= (1ull << 31)) return MPQ_ERR_SHAPE;
-    L->sched_words = (int32_t)sched_words_of(units, T);
+    if (sched_words_of(units, nz) >= (1ull << 31)) return MPQ_ERR_SHAPE;
+    L->sched_words = (int32_t)sched_words_of(units, nz);
 
     if (table) {
         table->assign((size_t)T, mpq_block{0, 0, 0, 0});
@@ -136,23 +137,36 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
                 row_last[nb] = (uint32_t)u;
         uint64_t slots = 0;
         for (int nb = 0; nb < NB; ++nb) {
-            const uint32_t nc = row_last[nb] - row_first[nb] + 1u;
+            const uint32_t nc = row_last[nb] - row_first[nb] + 1;
             row_slot[nb] = (uint32_t)slots;
             if (nc > 1) slots += nc;
         }
+        // stage descriptors: every non-zero block in block order
+        uint32_t* st = sched->data() + (size_t)units * DESC_WORDS;
         uint64_t seen[9] = {0}, k = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            const int b = bits[t];
+            if (!b) continue;
+            uint32_t* e = st + (size_t)k * STAGE_WORDS;
+            e[SW_CODE] = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
+            e[SW_SZ] = (uint32_t)(64u * k);
+            e[SW_KB_BITS] = (uint32_t)(t % KB) | ((uint32_t)b << 16);
+            e[SW_NB] = (uint32_t)(t / KB);
+            ++seen[b];
+            ++k;
+        }
+        uint64_t stage = 0;
         int64_t t = 0;
         for (int64_t u = 0; u < units; ++u) {
             const uint32_t t0 = bounds[(size_t)u], t1 = bounds[(size_t)u + 1];
             uint32_t* d = sched->data() + (size_t)u * DESC_WORDS;
-            for (; t < t0; ++t) { seen[bits[t]]++; k += bits[t] != 0; }
+            for (; t < t0; ++t) stage += bits[t] != 0;
+            uint64_t ns = 0;
+            for (uint32_t j = t0; j < t1; ++j) ns += bits[j] != 0;
             d[DW_T0] = t0;
             d[DW_T1] = t1;
-            d[DW_SZ] = (uint32_t)(64u * k);
-            for (int i = 0; i < 7; ++i) {
-                const int b = order[i];
-                d[DW_CODE + width_index(b)] = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
-            }
+            d[DW_S0] = (uint32_t)stage;
+            d[DW_NS] = (uint32_t)ns;
             const uint32_t ra = t0 / KB, rb = (t1 - 1) / KB;
             d[DW_A_SLOT] = row_slot[ra];
             d[DW_A_NC] = row_last[ra] - row_first[ra] + 1u;
@@ -160,11 +174,7 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
             d[DW_B_SLOT] = row_slot[rb];
             d[DW_B_NC] = row_last[rb] - row_first[rb] + 1u;
             d[DW_B_IDX] = (uint32_t)u - row_first[rb];
-            uint8_t* ib = reinterpret_cast<uint8_t*>(d + DW_BITS);
-            for (uint32_t j = 0; j < (uint32_t)DESC_INLINE_BITS && t0 + j < t1; ++j) ib[j] = bits[t0 + j];
         }
-        uint8_t* b8 = reinterpret_cast<uint8_t*>(sched->data() + (size_t)units * DESC_WORDS);
-        for (int64_t i = 0; i < T; ++i) b8[i] = bits[i];
     }
     return MPQ_OK;
 }
@@ -274,6 +284,7 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
 }
 std::atomic<uint64_t> g_decode_attr{0};
 std::atomic<uint64_t> g_decode_attr8{0};
+std::atomic<uint64_t> g_decode_attr16{0};
 std::atomic<uint64_t> g_decode_attr_f{0};
 std::atomic<uint64_t> g_decode_attr_g{0};
 std::atomic<uint64_t> g_prefill_attr{0};
@@ -480,7 +491,7 @@ DecodeParams decode_params(const mpq_layer* layer, const void* x_dev, int32_t M,
     DecodeParams dp{};
     dp.codes = static_cast<const uint8_t*>(layer->codes);
     dp.desc = layer->sched;
-    dp.bits8 = reinterpret_cast<const uint8_t*>(layer->sched + (size_t)layer->n_units * DESC_WORDS);
+    dp.stages = reinterpret_cast<const uint4*>(layer->sched + (size_t)layer->n_units * DESC_WORDS);
     dp.scales = layer->scales;
     dp.zeros = layer->zeros;
     dp.row_perm = layer->row_perm;
@@ -614,9 +625,10 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
         return MPQ_OK;
     }
 
-    e = ensure_smem_attr(k_decode<true>, (int)sizeof(DecSmem), g_decode_attr);
-    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<false>, (int)sizeof(DecSmem), g_decode_attr8);
-    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<true, true>, (int)sizeof(DecSmem), g_decode_attr_f);
+    e = ensure_smem_attr(k_decode<1>, (int)sizeof(DecSmem), g_decode_attr);
+    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<2>, (int)sizeof(DecSmem), g_decode_attr8);
+    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<4>, (int)sizeof(DecSmem), g_decode_attr16);
+    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<1, true>, (int)sizeof(DecSmem), g_decode_attr_f);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
     DecodeParams dp = decode_params(layer, x_dev, M, y_dev, w);
 
@@ -635,9 +647,11 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
     for (int m0 = 0; m0 < M; m0 += kMaxDecodeTokens) {
         dp.m0 = m0;
         dp.Mg = std::min(kMaxDecodeTokens, M - m0);
-        e = fused ? cudaLaunchKernelEx(&cfg, k_decode<true, true>, dp)
-            : dp.Mg == 1 ? cudaLaunchKernelEx(&cfg, k_decode<true>, dp)
-                         : cudaLaunchKernelEx(&cfg, k_decode<false>, dp);
+        // token groups of two: one for up to 2 tokens, two for 4, four for 8
+        e = fused ? cudaLaunchKernelEx(&cfg, k_decode<1, true>, dp)
+            : dp.Mg <= 2 ? cudaLaunchKernelEx(&cfg, k_decode<1>, dp)
+            : dp.Mg <= 4 ? cudaLaunchKernelEx(&cfg, k_decode<2>, dp)
+                         : cudaLaunchKernelEx(&cfg, k_decode<4>, dp);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
     }
     if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)

@@ -29,7 +29,8 @@ def block_cost(b):
 def restated_schedule(N, K, bits):
     """The schedule rules, restated: cost-prefix cuts (or, when there are no
     more non-zero blocks than runs, one non-zero block per run), empty runs
-    dropped, 32-word descriptors, then the width byte of every block."""
+    dropped, 32-word run descriptors, then a 4-word stage descriptor per
+    non-zero block in block order."""
     NB, KB = N // 64, K // 128
     T = NB * KB
     bits = np.asarray(bits, np.int64)
@@ -61,26 +62,24 @@ def restated_schedule(N, K, bits):
     for b in ORDER:
         seg_off[b] = off
         off += int((bits == b).sum()) * 1024 * b
-    words = DESC * U + (T + 3) // 4
+    words = DESC * U + 4 * len(nz)
     out = np.zeros(words, np.uint32)
     for u in range(U):
         t0, t1 = bounds[u], bounds[u + 1]
-        before = bits[:t0]
         d = out[DESC * u:DESC * (u + 1)]
         d[0], d[1] = t0, t1
-        d[2] = 64 * int((before != 0).sum())
-        for i, b in enumerate(ORDER):
-            d[3 + i] = seg_off[b] + 1024 * b * int((before == b).sum())
+        d[2] = int((bits[:t0] != 0).sum())
+        d[3] = int((bits[t0:t1] != 0).sum())
         ra, rb = t0 // KB, (t1 - 1) // KB
         d[10], d[11], d[12] = row_slot[ra], nc[ra], u - row_first[ra]
         d[13], d[14], d[15] = row_slot[rb], nc[rb], u - row_first[rb]
-        inl = np.zeros(64, np.uint8)
-        n = min(64, t1 - t0)
-        inl[:n] = bits[t0:t0 + n]
-        d[16:32] = inl.view(np.uint32)
-    b8 = np.zeros(4 * ((T + 3) // 4), np.uint8)
-    b8[:T] = bits
-    out[DESC * U:] = b8.view(np.uint32)
+    st = out[DESC * U:].reshape(-1, 4)
+    for k, t in enumerate(nz):
+        b = int(bits[t])
+        st[k, 0] = seg_off[b] + 1024 * b * int((bits[:t] == b).sum())
+        st[k, 1] = 64 * k
+        st[k, 2] = (t % KB) | (b << 16)
+        st[k, 3] = t // KB
     return out, bounds, row_slot, nc
 
 
@@ -104,7 +103,7 @@ def test_schedule_matches_restatement(name, L):
 
 
 def test_schedule_long_runs_and_all_zero():
-    # runs longer than the 64 inline widths (the per-block width bytes are used)
+    # runs of more than 32 non-zero blocks (several chunks of stage descriptors)
     rng = np.random.default_rng(3)
     N, K = 64 * 256, 128 * 1024          # 262144 blocks > 64 * MAX_UNITS
     bits = rng.choice(np.array([0, 1, 2, 3, 4], np.uint8), size=(N // 64) * (K // 128))
@@ -113,6 +112,8 @@ def test_schedule_long_runs_and_all_zero():
     want, bounds, _, _ = restated_schedule(N, K, bits)
     assert np.array_equal(got, want)
     assert max(np.diff(bounds)) > 64
+    d = got[:lay.n_units * DESC].reshape(-1, DESC)
+    assert d[:, 3].max() > 32
     # an all-zero layer still has runs (they write zeros)
     z = np.zeros(4 * 8, np.uint8)
     lz = B.plan(4 * 64, 8 * 128, z)
