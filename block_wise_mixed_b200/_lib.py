@@ -93,6 +93,8 @@ def lib():
         L.mpq_linear_noalloc.restype = ctypes.c_int
         L.mpq_noalloc_check.argtypes = [P]
         L.mpq_noalloc_check.restype = ctypes.c_int
+        L.mpq_fold_orders.argtypes = [i32, P, P, P]
+        L.mpq_fold_orders.restype = ctypes.c_int
         L.mpq_check.argtypes = [P, P]
         L.mpq_status_string.argtypes = [ctypes.c_int]
         L.mpq_status_string.restype = ctypes.c_char_p
@@ -311,6 +313,26 @@ def linear_host(layer: PackedLayer, x_host, y_host, ws, stream=None):
 
 def linear_host_workspace_size(layer: PackedLayer, M: int) -> int:
     return lib().mpq_linear_host_workspace_size(ctypes.byref(layer.c), M)
+
+
+def fold_orders(row_perm_a, col_perm_b, n: int) -> np.ndarray:
+    """mpq_fold_orders: the column order that lets layer B read layer A's
+    output in A's packed row order (A then runs with row_perm NULL)."""
+    a = None if row_perm_a is None else np.ascontiguousarray(row_perm_a, dtype=np.int32)
+    b = None if col_perm_b is None else np.ascontiguousarray(col_perm_b, dtype=np.int32)
+    out = np.zeros(n, np.int32)
+    _raise(lib().mpq_fold_orders(n, _np_ptr(a), _np_ptr(b), _np_ptr(out)), "mpq_fold_orders")
+    return out
+
+
+def with_orders(P: PackedLayer, row_perm=None, col_perm=None, keep_rows=True, keep_cols=True):
+    """A view of a packed layer for inference with other activation / output
+    orders (device int32 tensors or None): the packed buffers are shared."""
+    rp = P.row_perm if keep_rows else row_perm
+    cp = P.col_perm if keep_cols else col_perm
+    c = Layer(P.c.N, P.c.K, P.c.n_units, 0, P.c.codes, P.c.table, P.c.sched, P.c.scales, P.c.zeros,
+              rp.data_ptr() if rp is not None else None, cp.data_ptr() if cp is not None else None)
+    return PackedLayer(P.layout, P.codes, P.table, P.sched, P.scales, P.zeros, rp, cp, c)
 
 
 def check(ws, stream=None):

@@ -767,6 +767,17 @@ mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host, int32_t M
     return MPQ_OK;
 }
 
+mpq_status mpq_fold_orders(int32_t n, const int32_t* row_perm_a, const int32_t* col_perm_b,
+                           int32_t* out) {
+    if (n <= 0 || !out) return MPQ_ERR_ARG;
+    if ((row_perm_a && !perm_ok(row_perm_a, n)) || (col_perm_b && !perm_ok(col_perm_b, n)))
+        return MPQ_ERR_PERM;
+    std::vector<int32_t> inv((size_t)n);
+    for (int32_t i = 0; i < n; ++i) inv[(size_t)(row_perm_a ? row_perm_a[i] : i)] = i;
+    for (int32_t j = 0; j < n; ++j) out[j] = inv[(size_t)(col_perm_b ? col_perm_b[j] : j)];
+    return MPQ_OK;
+}
+
 mpq_status mpq_check(const void* ws, void* stream) {
     if (!ws) return MPQ_ERR_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

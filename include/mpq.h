@@ -291,6 +291,24 @@ mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t
  * array (memset, no allocation) so that the next call starts clean. */
 mpq_status mpq_noalloc_check(void* stream);
 
+/* Folds the output reordering of one layer into the input reordering of the
+ * next (SFMP abstract: reordering costs only "a small activation
+ * reordering overhead during inference"; this removes the output scatter of
+ * the first layer as well).  Host only.
+ *   Layer A (N_A outputs) was packed with row order row_perm_a; layer B
+ *   (K_B = N_A inputs) with column order col_perm_b.  Run A with a layer
+ *   whose row_perm is NULL: its y is then in A's packed row order,
+ *   y'[m][i] = y[m][row_perm_a[i]].  Run B on that y' (or on any elementwise
+ *   function of it) with col_perm = out, where
+ *     out[j] = inverse(row_perm_a)[col_perm_b[j]],  j < n,
+ *   so B gathers x'[m][j] = y'[m][out[j]] = y[m][col_perm_b[j]] -- the same
+ *   values, and the same result bit for bit, as the unfolded pair.
+ *   NULL for either order means identity; out (host, n int32) must not be
+ *   NULL.  Errors: ARG (n <= 0, out NULL), PERM (an order that is not a
+ *   bijection of 0..n-1). */
+mpq_status mpq_fold_orders(int32_t n, const int32_t* row_perm_a, const int32_t* col_perm_b,
+                           int32_t* out);
+
 /* Synchronizes `stream` and returns the device error word of `ws`: the first
  * device error of the mpq_linear calls on that workspace since it was
  * zero-filled or since the previous mpq_check, or of the last mpq_pack

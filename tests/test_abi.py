@@ -184,3 +184,29 @@ def test_misaligned_x_and_w_refused(lib):
     st = lib.mpq_pack(ctypes.byref(L), P(8), bits.ctypes.data_as(P), None, None, ctypes.byref(out),
                       P(256), ws_need, None)
     assert B.STATUS[st] == "MPQ_ERR_ARG"
+
+
+def test_fold_orders_host():
+    """mpq_fold_orders composes the inverse of layer A's row order with layer
+    B's column order; reading A's packed-order output through it gives B the
+    values its own order would gather."""
+    from block_wise_mixed_b200 import _lib
+    rng = np.random.default_rng(11)
+    n = 384
+    a = rng.permutation(n).astype(np.int32)
+    b = rng.permutation(n).astype(np.int32)
+    q = _lib.fold_orders(a, b, n)
+    y = rng.standard_normal((2, n))
+    assert np.array_equal(y[:, a][:, q], y[:, b])
+    # identities: NULL for either order
+    assert np.array_equal(_lib.fold_orders(None, b, n), b)
+    assert np.array_equal(_lib.fold_orders(a, None, n)[a], np.arange(n))
+    assert np.array_equal(_lib.fold_orders(None, None, n), np.arange(n))
+    # errors
+    bad = a.copy()
+    bad[0] = bad[1]
+    with pytest.raises(_lib.MpqError) as ei:
+        _lib.fold_orders(bad, b, n)
+    assert ei.value.name == "MPQ_ERR_PERM"
+    lib = _lib.lib()
+    assert _lib.STATUS[lib.mpq_fold_orders(0, None, None, None)] == "MPQ_ERR_ARG"

@@ -381,3 +381,32 @@ def test_linear_group_mixed_runs(mpq):
     ys = mpq.linear_group(Ps, x)
     for P, y in zip(Ps, ys):
         assert torch.equal(y, mpq.linear(P, x))
+
+
+# ---------------------------------------------------------------------------
+# Folding one layer's output order into the next layer's input order: layer A
+# runs without its row order (y in A's packed row order), layer B reads that
+# output through the composed column order (mpq_fold_orders); the result of
+# the pair is bit-identical to the unfolded pair, on the decode and the
+# tensor-core paths.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M", [1, 3, 40])
+def test_folded_layer_chain(mpq, M):
+    import torch
+    A = synth.make_layer("a", 512, 1024, 2.5, 8100, "random")
+    Bl = synth.make_layer("b", 256, 512, 3.0, 8200, "random")
+    PA, PB = pack_gpu(mpq, A), pack_gpu(mpq, Bl)
+    x = dev(synth.make_x(8300 + M, M, 1024))
+    # unfolded: A scatters y to the original order, B gathers through its order
+    ya = mpq.linear(PA, x)
+    yb = mpq.linear(PB, ya.to(torch.bfloat16).view(torch.int16))
+    # folded
+    q = torch.from_numpy(mpq.fold_orders(A.row_perm, Bl.col_perm, 512)).cuda()
+    PA_f = mpq.with_orders(PA, row_perm=None, keep_rows=False)
+    PB_f = mpq.with_orders(PB, col_perm=q, keep_cols=False)
+    ya_f = mpq.linear(PA_f, x)
+    yb_f = mpq.linear(PB_f, ya_f.to(torch.bfloat16).view(torch.int16))
+    torch.cuda.synchronize()
+    rp = torch.from_numpy(A.row_perm.astype(np.int64)).cuda()
+    assert torch.equal(ya_f, ya[:, rp])      # A's output in its packed row order
+    assert torch.equal(yb_f, yb)
