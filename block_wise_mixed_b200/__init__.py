@@ -5,7 +5,8 @@ fp16 scale/zero, bi-directional channel reordering) on NVIDIA B200.
 The computation lives in the C-ABI library ``libmpq.so`` (include/mpq.h); this
 package only marshals arguments to it.  ``synth`` draws seeded workloads.
 """
-from ._lib import (GROUP_MAX, Y_BF16, Y_F32, MpqError, PackedLayer, check, fold_orders, linear,  # noqa: F401
+from ._lib import (GROUP_MAX, Y_BF16, Y_F32, MpqError, PackedLayer, allocate_bits, check, fold_orders,  # noqa: F401
+                   linear,
                    linear_group, linear_group_workspace_size, linear_host, linear_host_workspace_size,
                    linear_timed, linear_typed_workspace_size, linear_workspace_size, pack, plan,
                    with_orders)

@@ -93,6 +93,10 @@ def lib():
         L.mpq_linear_noalloc.restype = ctypes.c_int
         L.mpq_noalloc_check.argtypes = [P]
         L.mpq_noalloc_check.restype = ctypes.c_int
+        L.mpq_allocate_bits_workspace_size.argtypes = [ctypes.c_int64]
+        L.mpq_allocate_bits_workspace_size.restype = sz
+        L.mpq_allocate_bits.argtypes = [ctypes.c_int64, P, ctypes.c_uint32, ctypes.c_uint64, P, P, P, sz, P]
+        L.mpq_allocate_bits.restype = ctypes.c_int
         L.mpq_fold_orders.argtypes = [i32, P, P, P]
         L.mpq_fold_orders.restype = ctypes.c_int
         L.mpq_check.argtypes = [P, P]
@@ -313,6 +317,28 @@ def linear_host(layer: PackedLayer, x_host, y_host, ws, stream=None):
 
 def linear_host_workspace_size(layer: PackedLayer, M: int) -> int:
     return lib().mpq_linear_host_workspace_size(ctypes.byref(layer.c), M)
+
+
+def allocate_bits(loss, allowed, budget: int, stream=None):
+    """mpq_allocate_bits: per-block widths (uint8 tensor) under a total-bits
+    budget from a device float32 loss table [n][8] (widths 0..6, 8).  Returns
+    (bits, iterations, total_bits)."""
+    import torch
+    n = loss.shape[0]
+    mask = 0
+    for b in allowed:
+        mask |= 1 << int(b)
+    bits = torch.empty(n, dtype=torch.uint8, device=loss.device)
+    info = torch.zeros(4, dtype=torch.int32, device=loss.device)
+    ws = torch.empty(max(lib().mpq_allocate_bits_workspace_size(n), 256), dtype=torch.uint8,
+                     device=loss.device)
+    lc = loss.contiguous()
+    _raise(lib().mpq_allocate_bits(n, lc.data_ptr(), mask, int(budget), bits.data_ptr(),
+                                   info.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "mpq_allocate_bits")
+    inf = info.cpu().numpy().view(np.uint32)
+    _raise(int(inf[3]), "mpq_allocate_bits (device)")
+    return bits, int(inf[0]), int(inf[1]) | (int(inf[2]) << 32)
 
 
 def fold_orders(row_perm_a, col_perm_b, n: int) -> np.ndarray:

@@ -12,6 +12,7 @@
 
 #include "../../include/mpq.h"
 #include "common.cuh"
+#include "k_alloc.cuh"
 #include "k_decode.cuh"
 #include "k_pack.cuh"
 #include "k_prefill.cuh"
@@ -765,6 +766,34 @@ mpq_status mpq_linear_host(const mpq_layer* layer, const void* x_host, int32_t M
     if (cudaMemcpyAsync(y_host, yb, (size_t)M * layer->N * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return MPQ_ERR_CUDA;
     return MPQ_OK;
+}
+
+size_t mpq_allocate_bits_workspace_size(int64_t n_blocks) {
+    if (n_blocks <= 0) return 0;
+    return round256((size_t)n_blocks * 8) + round256((size_t)n_blocks);
+}
+
+mpq_status mpq_allocate_bits(int64_t n_blocks, const float* loss_dev, uint32_t allowed,
+                             uint64_t budget, uint8_t* bits_dev, uint32_t* info_dev, void* ws,
+                             size_t ws_bytes, void* stream) {
+    if (n_blocks <= 0 || n_blocks > (1ll << 24) || !loss_dev || !bits_dev || !info_dev) return MPQ_ERR_ARG;
+    if (allowed == 0u || (allowed & ~0x17Fu)) return MPQ_ERR_ARG;   // widths 0..6 and 8
+    const int bmin = __builtin_ctz(allowed);
+    if (budget < (uint64_t)bmin * (uint64_t)n_blocks) return MPQ_ERR_ARG;
+    if (!ws || ws_bytes < mpq_allocate_bits_workspace_size(n_blocks) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255))
+        return MPQ_ERR_WORKSPACE;
+    AllocParams p{};
+    p.loss = loss_dev;
+    p.bits = bits_dev;
+    p.info = info_dev;
+    p.gkey = static_cast<unsigned long long*>(ws);
+    p.ginc = static_cast<uint8_t*>(ws) + round256((size_t)n_blocks * 8);
+    p.n = n_blocks;
+    p.budget = budget;
+    p.mask = allowed;
+    k_allocate_bits<<<1, ALLOC_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cuda_status(cudaGetLastError());
 }
 
 mpq_status mpq_fold_orders(int32_t n, const int32_t* row_perm_a, const int32_t* col_perm_b,

@@ -291,6 +291,40 @@ mpq_status mpq_linear_noalloc(const mpq_layer* layer, const void* x_dev, int32_t
  * array (memset, no allocation) so that the next call starts clean. */
 mpq_status mpq_noalloc_check(void* stream);
 
+/* Budgeted bit allocation: the bit map that mpq_plan / mpq_pack take, from
+ * per-block sensitivity surrogates under a global budget.  ScaleBITS
+ * abstract (bitwidth allocation under a memory budget by "a scalable
+ * approximation to the greedy algorithm") and summary page, "Approach" (a
+ * batched approximation to greedy knapsack allocation per 64x128 block) and
+ * "Key results" (16-36 search iterations against about 3e6 for classic
+ * greedy).  The library's reading: with a price lam per bit, each block
+ * takes argmin_b loss[t][b] + lam * b (fp64, the product rounded before the
+ * sum, ties to the smaller width); lam is bisected until the total fits the
+ * budget (from lo = 0 and hi = the largest per-bit saving over the smallest
+ * width, doubled while rounding leaves the total above the budget; until the
+ * total equals the budget, hi - lo <= hi * 2^-20, the midpoint equals an end,
+ * or 64 steps); the leftover is then filled in rounds, each taking the
+ * longest prefix of the next-width upgrades that save loss (saving per bit
+ * descending, block index ascending) whose increments fit.  On losses convex
+ * in the width this is the classic one-upgrade-at-a-time greedy's result.
+ *   n_blocks    blocks (1 .. 2^24), in any order the caller chooses (e.g. the
+ *               block ids of one layer, or all layers of a model).
+ *   loss_dev    device float [n_blocks][8]: the loss of each block at widths
+ *               0,1,2,3,4,5,6,8 (columns of widths not allowed are ignored).
+ *   allowed     bit b set = width b allowed (b in {0..6, 8}, at least one).
+ *   budget      total bits (sum of the widths); at least n_blocks times the
+ *               smallest allowed width.
+ *   bits_dev    device uint8 [n_blocks] (out): the widths.
+ *   info_dev    device uint32 [4] (out): search iterations (1 + bisection
+ *               steps + fill rounds), total bits (low word, high word),
+ *               status (MPQ_OK, or MPQ_ERR_NONFINITE for a non-finite loss).
+ *   ws          device workspace of mpq_allocate_bits_workspace_size bytes.
+ * One CTA runs the search (deterministic).  Host errors: ARG, WORKSPACE. */
+size_t mpq_allocate_bits_workspace_size(int64_t n_blocks);
+mpq_status mpq_allocate_bits(int64_t n_blocks, const float* loss_dev, uint32_t allowed,
+                             uint64_t budget, uint8_t* bits_dev, uint32_t* info_dev, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* Folds the output reordering of one layer into the input reordering of the
  * next (SFMP abstract: reordering costs only "a small activation
  * reordering overhead during inference"; this removes the output scatter of
