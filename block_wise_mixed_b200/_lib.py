@@ -67,47 +67,53 @@ def lib():
         if not os.path.exists(LIB_PATH):
             raise RuntimeError("libmpq.so not found at %s: build it with "
                                "block_wise_mixed_b200.build.build()" % LIB_PATH)
-        L = ctypes.CDLL(LIB_PATH)
-        P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
-        L.mpq_plan.argtypes = [i32, i32, P, ctypes.POINTER(Layout)]
-        L.mpq_plan_schedule.argtypes = [ctypes.POINTER(Layout), P, P]
-        L.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
-        L.mpq_pack_workspace_size.restype = sz
-        L.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
-        L.mpq_pack_timed.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P,
-                                     P, P]
-        L.mpq_linear_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
-        L.mpq_linear_workspace_size.restype = sz
-        L.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
-        L.mpq_linear_timed.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P, P, P]
-        L.mpq_linear_typed_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_int]
-        L.mpq_linear_typed_workspace_size.restype = sz
-        L.mpq_linear_typed.argtypes = [ctypes.POINTER(Layer), P, i32, P, ctypes.c_int, P, sz, P]
-        L.mpq_linear_group_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, i32]
-        L.mpq_linear_group_workspace_size.restype = sz
-        L.mpq_linear_group.argtypes = [ctypes.POINTER(Layer), i32, P, i32, P, P, sz, P]
-        L.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
-        L.mpq_linear_host_workspace_size.restype = sz
-        L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
-        L.mpq_linear_noalloc.argtypes = [ctypes.POINTER(Layer), P, i32, P, P]
-        L.mpq_linear_noalloc.restype = ctypes.c_int
-        L.mpq_noalloc_check.argtypes = [P]
-        L.mpq_noalloc_check.restype = ctypes.c_int
-        L.mpq_allocate_bits_workspace_size.argtypes = [ctypes.c_int64]
-        L.mpq_allocate_bits_workspace_size.restype = sz
-        L.mpq_allocate_bits.argtypes = [ctypes.c_int64, P, ctypes.c_uint32, ctypes.c_uint64, P, P, P, sz, P]
-        L.mpq_allocate_bits.restype = ctypes.c_int
-        L.mpq_fold_orders.argtypes = [i32, P, P, P]
-        L.mpq_fold_orders.restype = ctypes.c_int
-        L.mpq_check.argtypes = [P, P]
-        L.mpq_status_string.argtypes = [ctypes.c_int]
-        L.mpq_status_string.restype = ctypes.c_char_p
-        for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_typed",
-                  "mpq_linear_group", "mpq_linear_timed", "mpq_linear_host",
-                  "mpq_check"):
-            getattr(L, f).restype = ctypes.c_int
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+def load(path: str):
+    """A ctypes handle on a build of the library at `path`, with the C ABI's
+    argument and result types declared."""
+    L = ctypes.CDLL(path)
+    P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    L.mpq_plan.argtypes = [i32, i32, P, ctypes.POINTER(Layout)]
+    L.mpq_plan_schedule.argtypes = [ctypes.POINTER(Layout), P, P]
+    L.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
+    L.mpq_pack_workspace_size.restype = sz
+    L.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
+    L.mpq_pack_timed.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P,
+                                 P, P]
+    L.mpq_linear_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
+    L.mpq_linear_workspace_size.restype = sz
+    L.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
+    L.mpq_linear_timed.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P, P, P]
+    L.mpq_linear_typed_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_int]
+    L.mpq_linear_typed_workspace_size.restype = sz
+    L.mpq_linear_typed.argtypes = [ctypes.POINTER(Layer), P, i32, P, ctypes.c_int, P, sz, P]
+    L.mpq_linear_group_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, i32]
+    L.mpq_linear_group_workspace_size.restype = sz
+    L.mpq_linear_group.argtypes = [ctypes.POINTER(Layer), i32, P, i32, P, P, sz, P]
+    L.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
+    L.mpq_linear_host_workspace_size.restype = sz
+    L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
+    L.mpq_linear_noalloc.argtypes = [ctypes.POINTER(Layer), P, i32, P, P]
+    L.mpq_linear_noalloc.restype = ctypes.c_int
+    L.mpq_noalloc_check.argtypes = [P]
+    L.mpq_noalloc_check.restype = ctypes.c_int
+    L.mpq_allocate_bits_workspace_size.argtypes = [ctypes.c_int64]
+    L.mpq_allocate_bits_workspace_size.restype = sz
+    L.mpq_allocate_bits.argtypes = [ctypes.c_int64, P, ctypes.c_uint32, ctypes.c_uint64, P, P, P, sz, P]
+    L.mpq_allocate_bits.restype = ctypes.c_int
+    L.mpq_fold_orders.argtypes = [i32, P, P, P]
+    L.mpq_fold_orders.restype = ctypes.c_int
+    L.mpq_check.argtypes = [P, P]
+    L.mpq_status_string.argtypes = [ctypes.c_int]
+    L.mpq_status_string.restype = ctypes.c_char_p
+    for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_typed",
+              "mpq_linear_group", "mpq_linear_timed", "mpq_linear_host",
+              "mpq_check"):
+        getattr(L, f).restype = ctypes.c_int
+    return L
 
 
 def _np_ptr(a):

@@ -45,7 +45,17 @@
 
 namespace mpq {
 
+// Wait-test build (-DMPQ_WAIT_TEST, a separate library used only by the
+// timeout test, never the default build): waits give up after 2 ms, and the
+// producers arm their barriers without issuing any copy, so every first wait
+// runs out with nothing in flight.
+#ifdef MPQ_WAIT_TEST
+constexpr bool kWaitTest = true;
+constexpr uint64_t DEC_WAIT_NS = 2000000ull;
+#else
+constexpr bool kWaitTest = false;
 constexpr uint64_t DEC_WAIT_NS = 2000000000ull;
+#endif
 
 // Run descriptor: 32 words (the unused ones are zero).
 enum DescWord {
@@ -466,7 +476,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
     uint32_t qe_nb = 0, qe_bits = 0, qe_off = 0, qe_end = 0, qe_x = 0, qe_kb = 0;
     bool xq_ready = false;               // x' is written by the prologue kernel
     auto issue_more = [&]() {
-        while (q_tail - q_head < (uint32_t)DEC_SLOTS && next < ns && !aborted) {
+        while (q_tail - q_head < (uint32_t)DEC_SLOTS && next < ns && !aborted && !(kWaitTest && q_tail > 0)) {
             const int l = (int)(next & 31u);
             const uint32_t coff = __shfl_sync(0xffffffffu, cs.x, l);
             const uint32_t szo = __shfl_sync(0xffffffffu, cs.y, l);
@@ -489,10 +499,12 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
                 uint64_t* bar = &W.full[slot];
                 mbar_arrive_expect_tx(bar, FUSED_X ? size - xb : size);
                 uint8_t* dst = W.ring + off;
-                bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
-                bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
-                bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
-                if (!FUSED_X && xq_ready) issue_x(dst + 1024u * b + 256u, b, xo, bar);
+                if (!kWaitTest) {
+                    bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
+                    bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
+                    bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
+                    if (!FUSED_X && xq_ready) issue_x(dst + 1024u * b + 256u, b, xo, bar);
+                }
             }
             if (lane == (int)slot) {
                 qe_nb = nbs; qe_bits = b; qe_off = off; qe_end = start + size; qe_x = xo;
@@ -525,7 +537,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
             const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
-            if (lane == 0) issue_x(W.ring + ko + 1024u * kbits + 256u, kbits, kx, &W.full[slot]);
+            if (lane == 0 && !kWaitTest) issue_x(W.ring + ko + 1024u * kbits + 256u, kbits, kx, &W.full[slot]);
         }
     }
 

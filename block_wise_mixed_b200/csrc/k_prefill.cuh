@@ -362,7 +362,9 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                         const uint32_t bytes = (b0 ? 1024u * b0 + 256u : 0u) + (b1 ? 1024u * b1 + 256u : 0u);
                         mbar_arrive_expect_tx(&S.full_c[sc], bytes);
                         uint8_t* cst = S.c[sc];
-                        if (b0) {
+                        if (kWaitTest) {
+                            // wait-test build: armed, no copy; the consumers' waits run out
+                        } else if (b0) {
                             bulk_g2s(cst, p.codes + c0, 1024u * b0, &S.full_c[sc]);
                             bulk_g2s(cst + 16384, p.scales + s0, 128u, &S.full_c[sc]);
                             bulk_g2s(cst + 16384 + 128, p.zeros + s0, 128u, &S.full_c[sc]);
@@ -376,7 +378,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                         timed_out();
                     }
                 }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
+                if (!__shfl_sync(0xffffffffu, ok, 0) || kWaitTest) { stop = true; break; }
                 ++a;
             }
         }
@@ -384,7 +386,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     } else if (warp == PF_WARPS - 1) {
         // ------------------- producer of the activation tiles -----------------
         pdl_wait();   // x' comes from the prologue kernel
-        if (lane == 0) {
+        if (lane == 0 && !kWaitTest) {
             int bq = 0;   // half-k-block activation tiles issued
             for (int kb = 0; kb < KB && !S.abort_flag; ++kb) {
                 if ((bits_of(0, kb) | bits_of(1, kb)) == 0) continue;
