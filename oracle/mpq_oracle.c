@@ -31,7 +31,11 @@
  *   - RTN is asymmetric with the range widened to include 0; the fp16 scale is
  *     the SMALLEST fp16 value h with h*qmax >= (hi - lo); z = rne(-lo/s);
  *     q = clamp(rne(w/s) + z, 0, qmax); dequant = (q - z)*s;
- *   - bits are in {0,1,2,3,4,5,6,8}; a 0-bit block dequantizes to zero;
+ *   - bits are in {0,1,2,3,4,5,6,8,16}; a 0-bit block dequantizes to zero;
+ *     a 16-bit block keeps its bf16 weights unquantized ([TQ]: the
+ *     highest-scoring tiles stay at 16 bits while the rest are quantized);
+ *     its payload is the 64 x 128 bf16 bit patterns of the block, row-major,
+ *     and its scales/zeros are 1 and 0 (unused);
  *   - W'[i][j] = W[row_perm[i]][col_perm[j]]; blocks are defined on W';
  *   - the packed format ("format v1") is this library's own; see
  *     mpqo_pack below for the byte layout.
@@ -101,7 +105,7 @@ static uint16_t f16_from_small_int(int v)
 int mpqo_bits_valid(int b)
 {
     return b == 0 || b == 1 || b == 2 || b == 3 || b == 4 || b == 5 ||
-           b == 6 || b == 8;
+           b == 6 || b == 8 || b == 16;
 }
 
 /* A b-bit code is stored as one or two "pieces"; the low piece comes first.
@@ -125,7 +129,7 @@ int mpqo_pieces(int b, int widths[2])
 /* ------------------------------------------------------------------------ */
 
 /* Segments hold the payloads of all blocks of one bit width, in ascending
- * block id t = nb*KB + kb; segments are ordered b = 1,2,3,4,5,6,8.  Each
+ * block id t = nb*KB + kb; segments are ordered b = 1,2,3,4,5,6,8,16.  Each
  * payload is 1024*b bytes (64 rows x 128 codes x b bits).  table[4t..4t+3] =
  * {code_off, sz_off, bits, bit_prefix}: byte offset of the payload in the
  * codes buffer, index of the block's first scale/zero, the width, and the sum
@@ -139,14 +143,14 @@ int mpqo_plan(int32_t N, int32_t K, const uint8_t *bits, mpqo_layout *L,
     memset(L, 0, sizeof *L);
     L->N = N; L->K = K; L->NB = NB; L->KB = KB;
 
-    int64_t count[9] = {0};
+    int64_t count[17] = {0};
     for (int64_t t = 0; t < T; t++) {
         if (!mpqo_bits_valid(bits[t])) return MPQO_ERR_BITS;
         count[bits[t]]++;
     }
-    static const int order[7] = {1, 2, 3, 4, 5, 6, 8};
+    static const int order[8] = {1, 2, 3, 4, 5, 6, 8, 16};
     uint64_t off = 0;
-    for (int i = 0; i < 7; i++) {
+    for (int i = 0; i < 8; i++) {
         int b = order[i];
         L->seg_off[b] = off;
         L->seg_bytes[b] = (uint64_t)count[b] * 1024u * (uint64_t)b;
@@ -155,7 +159,7 @@ int mpqo_plan(int32_t N, int32_t K, const uint8_t *bits, mpqo_layout *L,
     L->codes_bytes = off;
     if (off >= ((uint64_t)1 << 32)) return MPQO_ERR_SHAPE;
 
-    uint64_t seen[9] = {0};
+    uint64_t seen[17] = {0};
     uint64_t nz = 0, prefix = 0;
     for (int64_t t = 0; t < T; t++) {
         int b = bits[t];
@@ -295,6 +299,27 @@ int mpqo_pack(int32_t N, int32_t K, const uint16_t *W, const uint8_t *bits,
             if (b == 0) continue;
             const uint32_t *e = table + 4 * t;
             uint8_t *payload = codes + e[0];
+            if (b == 16) {
+                /* passthrough: the bf16 weights, row-major; scale 1, zero 0;
+                 * every weight finite and within the binary16 range (the
+                 * tensor-core path multiplies in fp16) */
+                for (int r = 0; r < 64; r++) {
+                    int i = nb * 64 + r;
+                    int src_row = row_perm ? row_perm[i] : i;
+                    for (int j = 0; j < 128; j++) {
+                        int col = kb * 128 + j;
+                        int src_col = col_perm ? col_perm[col] : col;
+                        uint16_t wb = W[(int64_t)src_row * K + src_col];
+                        double v = mpqo_bf16_to_f64(wb);
+                        if (!isfinite(v)) return MPQO_ERR_NONFINITE;
+                        if (fabs(v) > 65504.0) return MPQO_ERR_RANGE;
+                        memcpy(payload + r * 256 + 2 * j, &wb, 2);
+                    }
+                    scales[e[1] + r] = 0x3C00;
+                    zeros[e[1] + r] = 0;
+                }
+                continue;
+            }
             int widths[2];
             int np = mpqo_pieces(b, widths);
             for (int r = 0; r < 64; r++) {
@@ -356,6 +381,14 @@ static void dequant_row_reordered(const mpqo_packed *P, int i, double *out)
         int b = (int)e[2];
         if (b == 0) {
             for (int j = 0; j < 128; j++) out[kb * 128 + j] = 0.0;
+            continue;
+        }
+        if (b == 16) {              /* passthrough: the stored bf16 weights */
+            for (int j = 0; j < 128; j++) {
+                uint16_t wb;
+                memcpy(&wb, P->codes + e[0] + r * 256 + 2 * j, 2);
+                out[kb * 128 + j] = mpqo_bf16_to_f64(wb);
+            }
             continue;
         }
         unpack_row(P->codes + e[0], b, r, q);

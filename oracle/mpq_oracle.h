@@ -24,7 +24,7 @@ enum {
 typedef struct {
     int32_t N, K, NB, KB;
     uint64_t codes_bytes, n_sz, bit_total;
-    uint64_t seg_off[9], seg_bytes[9];
+    uint64_t seg_off[17], seg_bytes[17];   /* index = bit width */
 } mpqo_layout;
 
 typedef struct {

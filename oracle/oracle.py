@@ -46,8 +46,8 @@ class _Layout(ctypes.Structure):
                 ("NB", ctypes.c_int32), ("KB", ctypes.c_int32),
                 ("codes_bytes", ctypes.c_uint64), ("n_sz", ctypes.c_uint64),
                 ("bit_total", ctypes.c_uint64),
-                ("seg_off", ctypes.c_uint64 * 9),
-                ("seg_bytes", ctypes.c_uint64 * 9)]
+                ("seg_off", ctypes.c_uint64 * 17),
+                ("seg_bytes", ctypes.c_uint64 * 17)]
 
 
 class _Packed(ctypes.Structure):

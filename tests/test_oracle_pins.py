@@ -173,12 +173,12 @@ def test_plan_closed_forms(oracle):
     rng = np.random.default_rng(3)
     N, K = 640, 1280
     T = (N // 64) * (K // 128)
-    bits = rng.choice(np.array([0, 1, 2, 3, 4, 5, 6, 8], np.uint8), T)
+    bits = rng.choice(np.array([0, 1, 2, 3, 4, 5, 6, 8, 16], np.uint8), T)
     lay, table = oracle.plan(N, K, bits)
     assert lay.codes_bytes == 1024 * int(bits.astype(np.int64).sum())
     assert lay.n_sz == 64 * int((bits > 0).sum())
     assert lay.bit_total == int(bits.astype(np.int64).sum())
-    order = [1, 2, 3, 4, 5, 6, 8]
+    order = [1, 2, 3, 4, 5, 6, 8, 16]
     off = 0
     for b in order:
         assert lay.seg_off[b] == off
@@ -198,7 +198,7 @@ def test_plan_closed_forms(oracle):
 
 @pytest.mark.parametrize("N,K,bits,err", [
     (63, 128, None, "SHAPE"), (64, 100, None, "SHAPE"), (0, 128, None, "SHAPE"),
-    (64, 128, [7], "BITS"), (64, 128, [9], "BITS")])
+    (64, 128, [7], "BITS"), (64, 128, [9], "BITS"), (64, 128, [15], "BITS"), (64, 128, [32], "BITS")])
 def test_plan_errors(oracle, N, K, bits, err):
     T = max(1, (N // 64) * (K // 128))
     b = np.array(bits if bits else [1] * T, np.uint8)
@@ -397,3 +397,66 @@ def test_pack_errors(oracle):
     b0 = bits.copy()
     b0[0] = 0
     oracle.pack(W, b0)
+
+
+# ---------------------------------------------------------------------------
+# 16-bit passthrough blocks (TileQuant abstract: the highest-scoring tiles
+# stay at 16 bits, the rest are quantized): the payload is the block's bf16
+# weights, row-major; scale 1 and zero 0; dequantized exactly.
+# ---------------------------------------------------------------------------
+def test_sixteen_bit_payload_is_the_weights(oracle):
+    L = _layer(N=128, K=256, seed=23)
+    bits = np.array([16, 8, 0, 16], np.uint8)           # 2 x 2 blocks
+    R = oracle.pack(L.W, bits, L.row_perm, L.col_perm)
+    Wp = L.W[L.row_perm][:, L.col_perm]                   # W' as bf16 bits
+    lay, table = oracle.plan(128, 256, bits)
+    for t in (0, 3):
+        nb, kb = divmod(t, 2)
+        off = int(table[t, 0])
+        block = Wp[64 * nb:64 * nb + 64, 128 * kb:128 * kb + 128]
+        got = R.codes[off:off + 16384].view(np.uint16).reshape(64, 128)
+        assert np.array_equal(got, block)                 # little-endian bf16, row-major
+        sz = int(table[t, 1])
+        assert np.all(R.scales[sz:sz + 64] == 0x3C00) and np.all(R.zeros[sz:sz + 64] == 0)
+    # segments: the 16-bit payloads come last, in block order
+    assert lay.seg_off[16] == lay.seg_bytes[8] and lay.seg_bytes[16] == 2 * 16384
+    assert int(table[0, 0]) == lay.seg_off[16] and int(table[3, 0]) == lay.seg_off[16] + 16384
+    # dequant: exactly the weights in 16-bit blocks
+    What = oracle.dequant(R)
+    Wf = synth.bf16_bits_to_f32(L.W).astype(np.float64)
+    rows16 = L.row_perm[0:64]
+    cols16 = L.col_perm[0:128]
+    assert np.array_equal(What[np.ix_(rows16, cols16)], Wf[np.ix_(rows16, cols16)])
+    rows16b = L.row_perm[64:128]
+    cols16b = L.col_perm[128:256]
+    assert np.array_equal(What[np.ix_(rows16b, cols16b)], Wf[np.ix_(rows16b, cols16b)])
+
+
+def test_all_sixteen_bit_layer_is_the_dense_product(oracle):
+    """A layer of 16-bit blocks only computes x W^T on the original weights."""
+    L = _layer(N=128, K=256, seed=29)
+    bits = np.full(4, 16, np.uint8)
+    R = oracle.pack(L.W, bits, L.row_perm, L.col_perm)
+    x = synth.make_x(29, 3, 256)
+    y, bnd = oracle.linear(R, x)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    Wf = synth.bf16_bits_to_f32(L.W).astype(np.float64)
+    ref = xf @ Wf.T
+    mag = np.abs(xf) @ np.abs(Wf).T
+    assert np.all(np.abs(y - ref) <= 1e-12 * mag)
+    assert np.allclose(bnd, np.abs(xf) @ np.abs(Wf).T, rtol=1e-12)
+
+
+def test_sixteen_bit_errors(oracle):
+    L = _layer(N=64, K=128, seed=31)
+    bits = np.array([16], np.uint8)
+    W = L.W.copy()
+    W[2, 3] = 0x7F80                                      # bf16 +inf
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.pack(W, bits)
+    assert ei.value.status == oracle.ERR_NONFINITE
+    W = L.W.copy()
+    W[2, 3] = synth.f32_to_bf16_bits(np.array([70000.0], np.float32))[0]   # beyond fp16
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.pack(W, bits)
+    assert ei.value.status == oracle.ERR_RANGE
