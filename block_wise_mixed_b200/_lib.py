@@ -39,7 +39,7 @@ class Layout(ctypes.Structure):
                 ("KB", ctypes.c_int32), ("n_units", ctypes.c_int32),
                 ("sched_words", ctypes.c_int32), ("codes_bytes", ctypes.c_uint64),
                 ("n_sz", ctypes.c_uint64), ("bit_total", ctypes.c_uint64),
-                ("seg_off", ctypes.c_uint64 * 9), ("seg_bytes", ctypes.c_uint64 * 9)]
+                ("seg_off", ctypes.c_uint64 * 17), ("seg_bytes", ctypes.c_uint64 * 17)]
 
 
 class Layer(ctypes.Structure):

@@ -122,10 +122,12 @@ static_assert(DEC_CTAS_PER_SM * (sizeof(DecSmem) + 1024) <= 228 * 1024, "decode 
 // largest stages: an 8-bit payload, or a 6-bit one with two activation variants
 static_assert(DEC_RING >= 8 * 1024 + 256 + DEC_MAX_TOKENS * XQD_VAR, "ring too small");
 static_assert(DEC_RING >= 6 * 1024 + 256 + 2 * DEC_MAX_TOKENS * XQD_VAR, "ring too small");
+static_assert(DEC_RING >= 8192 + DEC_MAX_TOKENS * (XQD_VAR + 128), "ring too small");
 
 __host__ __device__ constexpr int lo_width(int b) { return (b == 3) ? 2 : (b == 5 || b == 6) ? 4 : b; }
 __host__ __device__ constexpr int hi_width(int b) { return (b == 3 || b == 5) ? 1 : (b == 6) ? 2 : 0; }
-__host__ __device__ constexpr int variant_of(int p) { return p == 1 ? 0 : p == 2 ? 1 : p == 4 ? 2 : 3; }
+// activation variant of a piece width (16: the bf16 slice for passthrough blocks)
+__host__ __device__ constexpr int variant_of(int p) { return p == 1 ? 0 : p == 2 ? 1 : p == 4 ? 2 : p == 16 ? 4 : 3; }
 // index of width b in the descriptor's code offsets (1,2,3,4,5,6,8 -> 0..6)
 __host__ __device__ constexpr int width_index(int b) { return b == 8 ? 6 : b - 1; }
 
@@ -335,11 +337,82 @@ __device__ __forceinline__ void block_accumulate(const uint8_t* stage, const uin
     }
 }
 
+// bf16 MMA: D(16x8, fp32) += A(16x16, bf16) * B(16x8, bf16)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Half `half` (block rows 32 half .. +31) of a 16-bit passthrough block
+// (TileQuant abstract: the highest-scoring tiles stay at 16 bits): the bf16
+// weights times the bf16 activations, exact products, fp32 accumulation.  The
+// mma's k order is the lane's quarter of the row: for k-step ks quad lane t
+// holds columns 32t + 4ks .. +3, so each lane reads 64 contiguous bytes of a
+// row and of the activation slice (the bf16 variant is x' in column order).
+// mma rows: tile tt, row g = half row 16tt + g, row g + 8 = 16tt + g + 8;
+// columns = tokens 0..7.  The results go through the stage's fix-up area to
+// the lanes that own the rows in the quantized path (rows 8g + 2i + (t & 1)).
+template <int G>
+__device__ __forceinline__ void block_accumulate16(const uint8_t* stage, const uint8_t* xb, float* fix,
+                                                   int half, int g, int t, uint32_t Mg, float (&acc)[4][G]) {
+    uint32_t b[16];
+    {
+        const uint8_t* src = (uint32_t)g < Mg ? xb + g * XQD_VAR + 64 * t : nullptr;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 v = src ? reinterpret_cast<const uint4*>(src)[c] : make_uint4(0u, 0u, 0u, 0u);
+            b[4 * c] = v.x; b[4 * c + 1] = v.y; b[4 * c + 2] = v.z; b[4 * c + 3] = v.w;
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+        uint32_t a0[16], a1[16];
+        const uint8_t* r0 = stage + (16 * tt + g) * 256 + 64 * t;
+        const uint8_t* r1 = r0 + 8 * 256;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 v0 = reinterpret_cast<const uint4*>(r0)[c];
+            const uint4 v1 = reinterpret_cast<const uint4*>(r1)[c];
+            a0[4 * c] = v0.x; a0[4 * c + 1] = v0.y; a0[4 * c + 2] = v0.z; a0[4 * c + 3] = v0.w;
+            a1[4 * c] = v1.x; a1[4 * c + 1] = v1.y; a1[4 * c + 2] = v1.z; a1[4 * c + 3] = v1.w;
+        }
+        float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ks += 2) {
+            mma_bf16_16816(c, a0[2 * ks], a1[2 * ks], a0[2 * ks + 1], a1[2 * ks + 1], b[2 * ks], b[2 * ks + 1]);
+            mma_bf16_16816(d, a0[2 * ks + 2], a1[2 * ks + 2], a0[2 * ks + 3], a1[2 * ks + 3], b[2 * ks + 2],
+                           b[2 * ks + 3]);
+        }
+        const int ra = 16 * tt + g, rb = ra + 8;
+        const uint32_t t0 = 2u * t, t1 = 2u * t + 1u;
+        if (t0 < Mg) { fix[ra * Mg + t0] = c[0] + d[0]; fix[rb * Mg + t0] = c[2] + d[2]; }
+        if (t1 < Mg) { fix[ra * Mg + t1] = c[1] + d[1]; fix[rb * Mg + t1] = c[3] + d[3]; }
+    }
+    __syncwarp();
+    if ((g >> 2) == half) {   // this lane's rows 8g + 2i + (t & 1) lie in the half
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int rl = 8 * g + 2 * i + (t & 1) - 32 * half;
+#pragma unroll
+            for (int grp = 0; grp < G; ++grp) {
+                const uint32_t tok = 2u * grp + (uint32_t)(t >> 1);
+                if (tok < Mg) acc[i][grp] += fix[rl * Mg + tok];
+            }
+        }
+    }
+}
+
 // Stage layout in the ring (all parts 16-byte multiples):
 //   payload 1024*b | scales 128 | zeros 128 | activation variant of the low
 //   piece, 272 bytes per token | (split widths) the high piece's variant
 __host__ __device__ constexpr bool split_width(int b) { return hi_width(b) != 0; }
+//   16-bit block: one half (32 rows x 256 bytes) | the bf16 activation
+//   variant | a fix-up area of 32 rows x Mg fp32 (no scales or zeros)
 __device__ __forceinline__ uint32_t stage_bytes(uint32_t b, uint32_t Mg) {
+    if (b == 16) return 8192u + XQD_VAR * Mg + 128u * Mg;
     return 1024u * b + 256u + XQD_VAR * Mg * (split_width((int)b) ? 2u : 1u);
 }
 
@@ -413,6 +486,13 @@ __device__ __forceinline__ void fused_records(const DecodeParams& p, int4 cp, in
     v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
     v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
     v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
+    if (b == 16) {   // the bf16 slice, column order
+        *reinterpret_cast<uint2*>(rec + 8 * lane) =
+            make_uint2((uint32_t)xr[cp.x] | ((uint32_t)xr[cp.y] << 16), (uint32_t)xr[cp.z] | ((uint32_t)xr[cp.w] << 16));
+        fence_proxy_async_smem();
+        __syncwarp();
+        return;
+    }
     int X[4], T[3];
     float F;
     xqd_integerize(v, X, T, F);
@@ -460,7 +540,9 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
     bool aborted = false;            // a bounded wait ran out: stop computing
     // variant of piece width p's activation record: 1, 2, 4, 8 -> 0, 1, 2, 3;
     // the low piece of width b is variant (0x302221100 >> 4b) & 15
-    auto var_lo = [](uint32_t b) -> uint32_t { return (uint32_t)(0x302221100ull >> (4 * b)) & 15u; };
+    auto var_lo = [](uint32_t b) -> uint32_t {
+        return b == 16 ? 4u : (uint32_t)(0x302221100ull >> (4 * b)) & 15u;
+    };
     auto var_hi = [](uint32_t b) -> uint32_t { return (uint32_t)(0x001010000ull >> (4 * b)) & 15u; };
     auto issue_x = [&](uint8_t* dst, uint32_t b, uint32_t xo, uint64_t* bar) {
         bulk_g2s(dst, p.xq + xo, x_bytes, bar);
@@ -482,10 +564,12 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             const uint32_t szo = __shfl_sync(0xffffffffu, cs.y, l);
             const uint32_t kbb = __shfl_sync(0xffffffffu, cs.z, l);
             const uint32_t nbs = __shfl_sync(0xffffffffu, cs.w, l);
-            const uint32_t b = kbb >> 16;
+            const uint32_t b = (kbb >> 16) & 0xFFu;
+            const uint32_t hb = kbb >> 24;                 // 16-bit blocks: which row half
             const uint32_t xo = (kbb & 0xFFFFu) * rec_bytes + var_lo(b) * var_bytes + x_tok_off;
             const uint32_t xb = split_width((int)b) ? 2u * x_bytes : x_bytes;
-            const uint32_t size = 1024u * b + 256u + xb;   // stage_bytes(b, Mg)
+            const uint32_t pay = b == 16 ? 8192u : 1024u * b + 256u;   // payload (+ scales, zeros)
+            const uint32_t size = pay + xb + (b == 16 ? 128u * Mg : 0u);   // stage_bytes(b, Mg)
             if (q_head == q_tail) { r_head = 0; r_tail = 0; r_pos = 0; }   // empty ring: restart at 0
             // a stage never wraps: when the ring's tail end is too short, skip to 0
             const bool skip = r_pos + size > (uint32_t)DEC_RING;
@@ -497,17 +581,21 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
                 // the fused path writes activation records into the ring
                 if (FUSED_X) fence_proxy_async_smem();
                 uint64_t* bar = &W.full[slot];
-                mbar_arrive_expect_tx(bar, FUSED_X ? size - xb : size);
+                mbar_arrive_expect_tx(bar, FUSED_X ? pay : pay + xb);
                 uint8_t* dst = W.ring + off;
                 if (!kWaitTest) {
-                    bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
-                    bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
-                    bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
-                    if (!FUSED_X && xq_ready) issue_x(dst + 1024u * b + 256u, b, xo, bar);
+                    if (b == 16) {
+                        bulk_g2s(dst, p.codes + coff, 8192u, bar);
+                    } else {
+                        bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
+                        bulk_g2s(dst + 1024u * b, p.scales + szo, 128u, bar);
+                        bulk_g2s(dst + 1024u * b + 128u, p.zeros + szo, 128u, bar);
+                    }
+                    if (!FUSED_X && xq_ready) issue_x(dst + pay, b, xo, bar);
                 }
             }
             if (lane == (int)slot) {
-                qe_nb = nbs; qe_bits = b; qe_off = off; qe_end = start + size; qe_x = xo;
+                qe_nb = nbs; qe_bits = b | (hb << 8); qe_off = off; qe_end = start + size; qe_x = xo;
                 if (FUSED_X) qe_kb = kbb & 0xFFFFu;
             }
             r_head = start + size;
@@ -534,10 +622,11 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
     if (!FUSED_X) {
         for (uint32_t k = q_head; k < q_tail; ++k) {
             const uint32_t slot = k % DEC_SLOTS;
-            const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot);
+            const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot) & 0xFFu;
             const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
-            if (lane == 0 && !kWaitTest) issue_x(W.ring + ko + 1024u * kbits + 256u, kbits, kx, &W.full[slot]);
+            const uint32_t kpay = kbits == 16 ? 8192u : 1024u * kbits + 256u;
+            if (lane == 0 && !kWaitTest) issue_x(W.ring + ko + kpay, kbits, kx, &W.full[slot]);
         }
     }
 
@@ -564,7 +653,8 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             const uint32_t slot = q_head % DEC_SLOTS;
             const uint32_t fnb = __shfl_sync(0xffffffffu, qe_nb, slot);
             if (fnb != nb) break;           // the next block is in a later row
-            const uint32_t fb = __shfl_sync(0xffffffffu, qe_bits, slot);
+            const uint32_t fbh = __shfl_sync(0xffffffffu, qe_bits, slot);
+            const uint32_t fb = fbh & 0xFFu;
             const uint32_t foff = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t fend = __shfl_sync(0xffffffffu, qe_end, slot);
             if (!aborted) {
@@ -576,7 +666,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             }
             if (!aborted) {
                 const uint8_t* stage = W.ring + foff;
-                uint8_t* xs = W.ring + foff + 1024u * fb + 256u;
+                uint8_t* xs = W.ring + foff + (fb == 16 ? 8192u : 1024u * fb + 256u);
                 if (FUSED_X) {
                     const uint32_t kb = __shfl_sync(0xffffffffu, qe_kb, slot);
                     const int4 cp = (kb == cp_kb) ? cp_pref : fused_cols(p, kb, lane);
@@ -584,7 +674,10 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
                 }
                 const uint8_t* xh = xs + x_bytes;
                 const uint8_t* z32 = reinterpret_cast<const uint8_t*>(W.zero32);
-                switch (fb) {
+                if (fb == 16)
+                    block_accumulate16<G>(stage, xs, reinterpret_cast<float*>(xs + x_bytes), (int)(fbh >> 8), g, t,
+                                          Mg, acc);
+                else switch (fb) {
                     case 1: block_accumulate<1, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
                     case 2: block_accumulate<2, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
                     case 3: block_accumulate<3, G>(stage, xs, xh, z32, g, t, Mg, acc); break;

@@ -115,6 +115,37 @@ k_pack(PackParams p) {
             const mpq_block e = p.table[(size_t)nb * KB + kb];
             const int b = (int)e.bits;
             if (b == 0) continue;
+            if (b == 16) {
+                // passthrough (TileQuant abstract: the highest-scoring tiles
+                // stay at 16 bits): the row's bf16 weights, scale 1, zero 0;
+                // finite and within the fp16 range (the tensor-core path)
+                const int c0 = kb * 128 + 4 * lane;
+                uint16_t wb[4];
+                bool finite = true, in_range = true;
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const int c = p.col_perm ? (int)cperm[c0 + e4] : c0 + e4;
+                    wb[e4] = row[c];
+                    const float v = __uint_as_float(((uint32_t)wb[e4]) << 16);
+                    finite &= isfinite(v);
+                    in_range &= fabsf(v) <= 65504.f;
+                }
+                if (!__all_sync(0xffffffffu, finite)) {
+                    if (lane == 0) set_error(p.err, MPQ_ERR_NONFINITE);
+                    continue;
+                }
+                if (!__all_sync(0xffffffffu, in_range)) {
+                    if (lane == 0) set_error(p.err, MPQ_ERR_RANGE);
+                    continue;
+                }
+                *reinterpret_cast<uint2*>(p.codes + e.code_off + (uint32_t)r * 256u + 8u * lane) =
+                    make_uint2((uint32_t)wb[0] | ((uint32_t)wb[1] << 16), (uint32_t)wb[2] | ((uint32_t)wb[3] << 16));
+                if (lane == 0) {
+                    p.scales[e.sz_off + r] = 0x3C00u;
+                    p.zeros[e.sz_off + r] = 0u;
+                }
+                continue;
+            }
             // gather this lane's 4 contiguous columns j = 4*lane .. 4*lane+3
             float w[4];
             const int c0 = kb * 128 + 4 * lane;

@@ -169,6 +169,36 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int kc) {
                       (((kc & 7) ^ (r & 7)) << 4));
 }
 
+// A 16-bit passthrough block (TileQuant abstract: the highest-scoring tiles
+// stay at 16 bits): groups [g0, g0+4) of row rr, read straight from the
+// block's bf16 payload in global memory (16 bytes per group), converted to
+// fp16 (exact for |w| in the fp16 normal range; the pack limits |w| to
+// 65504) and stored in the tile's column order.
+__device__ __forceinline__ void passthrough_row_part(const uint8_t* blk, int rr, int g0, uint8_t* a_tile, int r) {
+    const int sw = (g0 & 8) ? 2 : 0;
+    uint4 v[4];
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi)
+        v[gi] = __ldg(reinterpret_cast<const uint4*>(blk + rr * 256 + 16 * (g0 + (gi ^ sw))));
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) {
+        const uint32_t u[4] = {v[gi].x, v[gi].y, v[gi].z, v[gi].w};
+        float f[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            f[2 * c] = __uint_as_float(u[c] << 16);
+            f[2 * c + 1] = __uint_as_float(u[c] & 0xFFFF0000u);
+        }
+        // position pair j of the chunk holds columns (j, j + 4)
+        uint4 w;
+        w.x = h2_bits(__floats2half2_rn(f[0], f[4]));
+        w.y = h2_bits(__floats2half2_rn(f[1], f[5]));
+        w.z = h2_bits(__floats2half2_rn(f[2], f[6]));
+        w.w = h2_bits(__floats2half2_rn(f[3], f[7]));
+        *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + (gi ^ sw))) = w;
+    }
+}
+
 // Dequantizes groups [g0, g0+4) (8 codes each) of row rr of one block of
 // width B into the A tile row r: w_hat = (q - z) * s in fp16.  A warp covers
 // 8 whole rows (lane = row * 4 + quarter), so the lanes' code bytes are one
@@ -359,17 +389,25 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                     const uint32_t pc = (uint32_t)(a / PF_C_STAGES) & 1u;
                     ok = !S.abort_flag && mbar_wait_bounded(&S.empty_c[sc], pc ^ 1u, DEC_WAIT_NS);
                     if (ok) {
-                        const uint32_t bytes = (b0 ? 1024u * b0 + 256u : 0u) + (b1 ? 1024u * b1 + 256u : 0u);
-                        mbar_arrive_expect_tx(&S.full_c[sc], bytes);
+                        // 16-bit blocks are read by the dequantizing warps
+                        // themselves: the stage carries their payload offsets
+                        const uint32_t q0 = (b0 && b0 != 16) ? b0 : 0u, q1 = (b1 && b1 != 16) ? b1 : 0u;
+                        const uint32_t bytes = (q0 ? 1024u * q0 + 256u : 0u) + (q1 ? 1024u * q1 + 256u : 0u);
                         uint8_t* cst = S.c[sc];
+                        if (b0 == 16) *reinterpret_cast<uint32_t*>(cst + 16384) = c0;
+                        if (b1 == 16) *reinterpret_cast<uint32_t*>(cst + 16384 + 256) = c1;
+                        // those generic writes, and the ones of the stage's earlier
+                        // uses, come before this use's bulk copies
+                        fence_proxy_async_smem();
+                        mbar_arrive_expect_tx(&S.full_c[sc], bytes);
                         if (kWaitTest) {
                             // wait-test build: armed, no copy; the consumers' waits run out
-                        } else if (b0) {
+                        } else if (q0) {
                             bulk_g2s(cst, p.codes + c0, 1024u * b0, &S.full_c[sc]);
                             bulk_g2s(cst + 16384, p.scales + s0, 128u, &S.full_c[sc]);
                             bulk_g2s(cst + 16384 + 128, p.zeros + s0, 128u, &S.full_c[sc]);
                         }
-                        if (b1) {
+                        if (q1 && !kWaitTest) {
                             bulk_g2s(cst + 8192, p.codes + c1, 1024u * b1, &S.full_c[sc]);
                             bulk_g2s(cst + 16384 + 256, p.scales + s1, 128u, &S.full_c[sc]);
                             bulk_g2s(cst + 16384 + 384, p.zeros + s1, 128u, &S.full_c[sc]);
@@ -472,6 +510,10 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                         *reinterpret_cast<uint4*>(a_tile + sw128_chunk(r, g0 + gi)) = zero;
                     break;
                 }
+                case 16:
+                    passthrough_row_part(p.codes + *reinterpret_cast<const uint32_t*>(cst + 16384 + h * 256), rr, g0,
+                                         a_tile, r);
+                    break;
                 case 1: dequant_row_part<1>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
                 case 2: dequant_row_part<2>(cst + h * 8192, scz, rr, g0, a_tile, r); break;
                 case 3: dequant_row_part<3>(cst + h * 8192, scz, rr, g0, a_tile, r); break;

@@ -130,13 +130,16 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
 //   [d = 0..2][t = 0..3][j = 0..3][hf = 0, 1][b = 0..3] s8: digit d of X at
 //   column kappa -- for quad lane t and mma column d, the 32 bytes are its
 //   B-fragment registers of the four k-tiles in order;
-//   then T_0, T_1, T_2 (int32) and F (float).
-// so one variant of a token group is one contiguous run of 400*Mg bytes.
+//   then T_0, T_1, T_2 (int32) and F (float);
+// and variant 4, for 16-bit passthrough blocks: the slice's 128 bf16 values
+// in column order (the first 256 of its 400 bytes).  One variant of a token
+// group is one contiguous run of 400*Mg bytes.
 // Block 0 also clears the decode kernel's per-block-row counters.
 // ---------------------------------------------------------------------------
 constexpr int XQD_DIGITS = 3;
 constexpr int XQD_VAR = XQD_DIGITS * 128 + 16;   // one variant of one token: digits, T_d, F
-constexpr int XQD_REC = 4 * XQD_VAR;
+constexpr int XQD_VARIANTS = 5;                  // p = 1, 2, 4, 8, and the bf16 slice
+constexpr int XQD_REC = XQD_VARIANTS * XQD_VAR;
 constexpr float XQD_XMAX = 8355711.f;            // 127 * (1 + 256 + 65536): three s8 digits
 
 __host__ __device__ __forceinline__ int xqd_col(int v, int kappa) {
@@ -272,6 +275,9 @@ __global__ void __launch_bounds__(XPREP_THREADS, 8) k_xprep_decode(XprepParams p
                 reinterpret_cast<const uint4*>(rs)[lane];
         __syncwarp();
     }
+    // variant 4: the bf16 slice in column order
+    *reinterpret_cast<uint2*>(rec + (size_t)4 * p.M * XQD_VAR + 8 * lane) =
+        make_uint2((uint32_t)xr[cp.x] | ((uint32_t)xr[cp.y] << 16), (uint32_t)xr[cp.z] | ((uint32_t)xr[cp.w] << 16));
 }
 
 }  // namespace mpq

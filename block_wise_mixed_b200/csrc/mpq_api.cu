@@ -31,7 +31,9 @@ constexpr int kPackRowsPerCta = 1;
 
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline bool bits_ok(int b) { return b == 0 || b == 1 || b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8; }
+inline bool bits_ok(int b) {
+    return b == 0 || b == 1 || b == 2 || b == 3 || b == 4 || b == 5 || b == 6 || b == 8 || b == 16;
+}
 
 // Estimated cost of one block for the decode schedule, in bytes: what it
 // streams (payload, scales/zeros, one activation variant) plus a stand-in
@@ -39,6 +41,7 @@ inline bool bits_ok(int b) { return b == 0 || b == 1 || b == 2 || b == 3 || b ==
 // widths (3, 5, 6) make two passes.  Zero-bit blocks only cost bookkeeping.
 inline uint64_t block_cost(int b) {
     static const uint32_t work[9] = {0, 2048, 2048, 4096, 2304, 4352, 4352, 0, 2560};
+    if (b == 16) return 16384u + 256u + 272u + 2048u;   // two halves, bf16 mma
     return b == 0 ? 32u : 1024u * (uint64_t)b + 256u + 272u + work[b];
 }
 
@@ -57,12 +60,12 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
     const int64_t T = (int64_t)NB * KB;
     std::memset(L, 0, sizeof *L);
     L->N = N; L->K = K; L->NB = NB; L->KB = KB;
-    uint64_t count[9] = {0};
+    uint64_t count[17] = {0};
     for (int64_t t = 0; t < T; ++t) {
         if (!bits_ok(bits[t])) return MPQ_ERR_BITS;
         ++count[bits[t]];
     }
-    static const int order[7] = {1, 2, 3, 4, 5, 6, 8};
+    static const int order[8] = {1, 2, 3, 4, 5, 6, 8, 16};
     uint64_t off = 0;
     for (int b : order) {
         L->seg_off[b] = off;
@@ -71,10 +74,11 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
     }
     L->codes_bytes = off;
     if (off >= (1ull << 32)) return MPQ_ERR_SHAPE;
-    uint64_t nz = 0, total = 0;
-    for (int64_t t = 0; t < T; ++t) total += bits[t], nz += bits[t] != 0;
+    uint64_t nz = 0, total = 0, n16 = 0;
+    for (int64_t t = 0; t < T; ++t) total += bits[t], nz += bits[t] != 0, n16 += bits[t] == 16;
     L->n_sz = 64u * nz;
     L->bit_total = total;
+    const uint64_t n_stages = nz + n16;   // a 16-bit block streams as two halves
 
     // decode runs: cut the cost prefix into about equal parts, drop empty runs
     std::vector<uint64_t> pre((size_t)T + 1, 0);
@@ -106,12 +110,12 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
     bounds.push_back((uint32_t)T);
     const int64_t units = (int64_t)bounds.size() - 1;
     L->n_units = (int32_t)units;
-    if (sched_words_of(units, nz) >= (1ull << 31)) return MPQ_ERR_SHAPE;
-    L->sched_words = (int32_t)sched_words_of(units, nz);
+    if (sched_words_of(units, n_stages) >= (1ull << 31)) return MPQ_ERR_SHAPE;
+    L->sched_words = (int32_t)sched_words_of(units, n_stages);
 
     if (table) {
         table->assign((size_t)T, mpq_block{0, 0, 0, 0});
-        uint64_t seen[9] = {0}, k = 0, bp = 0;
+        uint64_t seen[17] = {0}, k = 0, bp = 0;
         for (int64_t t = 0; t < T; ++t) {
             const int b = bits[t];
             mpq_block& e = (*table)[(size_t)t];
@@ -142,28 +146,34 @@ mpq_status make_plan(int32_t N, int32_t K, const uint8_t* bits, mpq_layout* L,
             row_slot[nb] = (uint32_t)slots;
             if (nc > 1) slots += nc;
         }
-        // stage descriptors: every non-zero block in block order
+        // stage descriptors: every non-zero block in block order (a 16-bit
+        // block twice: rows 0..31, then rows 32..63)
         uint32_t* st = sched->data() + (size_t)units * DESC_WORDS;
-        uint64_t seen[9] = {0}, k = 0;
+        uint64_t seen[17] = {0}, k = 0, si = 0;
         for (int64_t t = 0; t < T; ++t) {
             const int b = bits[t];
             if (!b) continue;
-            uint32_t* e = st + (size_t)k * STAGE_WORDS;
-            e[SW_CODE] = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
-            e[SW_SZ] = (uint32_t)(64u * k);
-            e[SW_KB_BITS] = (uint32_t)(t % KB) | ((uint32_t)b << 16);
-            e[SW_NB] = (uint32_t)(t / KB);
+            const uint32_t code = (uint32_t)(L->seg_off[b] + seen[b] * 1024u * (uint64_t)b);
+            for (uint32_t half = 0; half < (b == 16 ? 2u : 1u); ++half) {
+                uint32_t* e = st + (size_t)si * STAGE_WORDS;
+                e[SW_CODE] = code + half * 8192u;
+                e[SW_SZ] = (uint32_t)(64u * k);
+                e[SW_KB_BITS] = (uint32_t)(t % KB) | ((uint32_t)b << 16) | (half << 24);
+                e[SW_NB] = (uint32_t)(t / KB);
+                ++si;
+            }
             ++seen[b];
             ++k;
         }
+        auto stages_of = [&](int b) -> uint64_t { return b == 0 ? 0u : b == 16 ? 2u : 1u; };
         uint64_t stage = 0;
         int64_t t = 0;
         for (int64_t u = 0; u < units; ++u) {
             const uint32_t t0 = bounds[(size_t)u], t1 = bounds[(size_t)u + 1];
             uint32_t* d = sched->data() + (size_t)u * DESC_WORDS;
-            for (; t < t0; ++t) stage += bits[t] != 0;
+            for (; t < t0; ++t) stage += stages_of(bits[t]);
             uint64_t ns = 0;
-            for (uint32_t j = t0; j < t1; ++j) ns += bits[j] != 0;
+            for (uint32_t j = t0; j < t1; ++j) ns += stages_of(bits[j]);
             d[DW_T0] = t0;
             d[DW_T1] = t1;
             d[DW_S0] = (uint32_t)stage;

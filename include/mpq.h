@@ -24,34 +24,41 @@
  *   W is N x K (out x in, nn.Linear layout), bf16, row-major.  With
  *   permutations P_r (N) and P_c (K), W'[i][j] = W[P_r[i]][P_c[j]].
  *   Block (nb, kb) of W' is rows 64nb..64nb+63, columns 128kb..128kb+127;
- *   block id t = nb*KB + kb; each block has bits[t] in {0,1,2,3,4,5,6,8}.
+ *   block id t = nb*KB + kb; each block has bits[t] in {0,1,2,3,4,5,6,8,16}.
  *   Each block row is one RTN group of 128 weights:
  *     lo = min(min w, 0), hi = max(max w, 0), d = hi - lo, qmax = 2^b - 1,
  *     s  = smallest fp16 h with h*qmax >= d  (s = 1 if d == 0),
  *     z  = rne(-lo / s) (an integer in [0, qmax], stored as fp16),
  *     q  = clamp(rne(w / s) + z, 0, qmax),   w_hat = (q - z) * s.
- *   A 0-bit block has no codes and dequantizes to zero.
+ *   A 0-bit block has no codes and dequantizes to zero.  A 16-bit block keeps
+ *   its bf16 weights (w_hat = w; TileQuant abstract: the highest-scoring
+ *   tiles stay at 16 bits); its weights must be finite and |w| <= 65504.
  *   y[m][P_r[i]] = sum_j x[m][P_c[j]] * w_hat'[i][j]   (y is fp32).
  *
  * Packed format v1 (the library's own; the pages name no layout):
- *   codes   -- segments for b = 1,2,3,4,5,6,8 in that order, each holding the
- *              payloads of all b-bit blocks in ascending t.  A payload is
+ *   codes   -- segments for b = 1,2,3,4,5,6,8,16 in that order, each holding
+ *              the payloads of all b-bit blocks in ascending t.  A payload is
  *              1024*b bytes: the code's "pieces" (1->[1], 2->[2], 3->[2,1],
  *              4->[4], 5->[4,1], 6->[4,2], 8->[8]; q = lo | hi << width(lo)),
  *              low piece first; a p-bit piece is 64 rows x 16p bytes,
  *              row-major; in a row, code j sits in little-endian 32-bit word
- *              j/(32/p) at bit (j%(32/p))*p.
+ *              j/(32/p) at bit (j%(32/p))*p.  A 16-bit payload is the
+ *              block's 64 x 128 bf16 bit patterns, row-major.
  *   scales, zeros -- fp16 bit patterns, 64 per non-zero block, in ascending t;
- *              row r of block t is at table[t].sz_off + r.
+ *              row r of block t is at table[t].sz_off + r (1 and 0 for a
+ *              16-bit block).
  *   table   -- one mpq_block per block (ascending t).
  *   sched   -- the decode schedule, sched_words 32-bit words: the blocks are
  *              cut into n_units row-major runs [t0, t1) of about equal
  *              estimated cost (bytes streamed plus decode work by width),
  *              one per decode warp.  Run u has a 32-word descriptor at word
- *              32u: t0, t1, the scale/zero index and the code offset of its
- *              first block of each width, the partial-sum slots of its
- *              first and last block rows, and the widths of its first 64
- *              blocks.  After the descriptors: one byte per block, its width.
+ *              32u: t0, t1, the index of its first stage and its number of
+ *              stages, and the partial-sum slots of its first and last block
+ *              rows (the other words are 0).  After the descriptors, 4 words
+ *              per stage, in block order: payload byte offset, scale/zero
+ *              index, block column | width << 16 | half << 24, block row.  A
+ *              quantized block is one stage; a 16-bit block is two (its rows
+ *              0..31 and 32..63, half 0 and 1).
  *
  * Conventions:
  *   - The caller owns every buffer.  The library allocates no device memory
@@ -86,10 +93,11 @@ typedef enum {
     MPQ_OK = 0,
     MPQ_ERR_ARG = 1,        /* NULL pointer or inconsistent argument        */
     MPQ_ERR_SHAPE = 2,      /* N % 64, K % 128, N or K <= 0, M < 0, too big  */
-    MPQ_ERR_BITS = 3,       /* a bit width outside {0,1,2,3,4,5,6,8}         */
+    MPQ_ERR_BITS = 3,       /* a bit width outside {0,1,2,3,4,5,6,8,16}      */
     MPQ_ERR_PERM = 4,       /* a permutation that is not a bijection         */
     MPQ_ERR_NONFINITE = 5,  /* NaN/Inf in W (device-detected)               */
-    MPQ_ERR_RANGE = 6,      /* no fp16 scale, or qmax*s > 65504 (device)    */
+    MPQ_ERR_RANGE = 6,      /* no fp16 scale, qmax*s > 65504, or a 16-bit
+                               block weight beyond +-65504 (device)          */
     MPQ_ERR_WORKSPACE = 7,  /* workspace missing or too small               */
     MPQ_ERR_CUDA = 8,       /* a CUDA call failed                           */
     MPQ_ERR_TIMEOUT = 9     /* a bounded device wait ran out (device)       */
@@ -105,7 +113,7 @@ typedef enum {
 typedef struct {
     uint32_t code_off;    /* byte offset of the payload in `codes` (0 if 0-bit) */
     uint32_t sz_off;      /* index of the block's row 0 in scales/zeros          */
-    uint32_t bits;        /* 0,1,2,3,4,5,6 or 8                                  */
+    uint32_t bits;        /* 0,1,2,3,4,5,6,8 or 16                               */
     uint32_t bit_prefix;  /* sum of bits of all blocks with a smaller id        */
 } mpq_block;
 
@@ -117,8 +125,8 @@ typedef struct {
     uint64_t codes_bytes;    /* = 1024 * bit_total                              */
     uint64_t n_sz;           /* = 64 * number of non-zero blocks                */
     uint64_t bit_total;      /* sum of the per-block bits                       */
-    uint64_t seg_off[9];     /* byte offset of segment b (index = bit width)    */
-    uint64_t seg_bytes[9];   /* bytes of segment b ([0] and [7] are 0)          */
+    uint64_t seg_off[17];    /* byte offset of segment b (index = bit width)    */
+    uint64_t seg_bytes[17];  /* bytes of segment b (0 for unused widths)         */
 } mpq_layout;
 
 /* A packed layer: device pointers to caller-owned buffers of the sizes in

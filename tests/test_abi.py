@@ -32,7 +32,7 @@ def test_status_strings(lib):
 
 def test_struct_sizes():
     assert ctypes.sizeof(B.Block) == 16
-    assert ctypes.sizeof(B.Layout) == 4 * 6 + 8 * 3 + 8 * 18
+    assert ctypes.sizeof(B.Layout) == 4 * 6 + 8 * 3 + 8 * 34     # seg_off, seg_bytes: index = width 0..16
     assert ctypes.sizeof(B.Layer) == 16 + 7 * 8
 
 

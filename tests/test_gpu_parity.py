@@ -95,7 +95,7 @@ def test_linear_configs(mpq, oracle, cfg, M):
     assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
 
 
-@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 6, 8, 16])
 def test_single_block_each_width(mpq, oracle, b):
     L = synth.make_layer("blk", 64, 128, float(b), 900 + b, "random", allowed=(b,))
     assert np.all(L.bits == b)
@@ -410,3 +410,37 @@ def test_folded_layer_chain(mpq, M):
     rp = torch.from_numpy(A.row_perm.astype(np.int64)).cuda()
     assert torch.equal(ya_f, ya[:, rp])      # A's output in its packed row order
     assert torch.equal(yb_f, yb)
+
+
+
+# ---------------------------------------------------------------------------
+# TileQuant-style two-level tiles (TileQuant abstract: within each
+# projection's retention budget the highest-scoring tiles stay at 16 bits and
+# the rest use 8 bits): 16-bit passthrough blocks beside 8-bit ones, and
+# beside every quantized width; decode (M <= 16) and tensor-core paths.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("allowed,avg,perm", [((8, 16), 8.8, "saliency"), ((8, 16), 9.6, "identity"),
+                                              ((0, 1, 2, 3, 4, 5, 6, 8, 16), 4.0, "random")])
+def test_sixteen_bit_tiles(mpq, oracle, allowed, avg, perm):
+    L = synth.make_layer("tq", 1024, 2048, avg, 9100 + int(10 * avg), perm, allowed=allowed)
+    if not (L.bits == 16).any():          # a low average draws none: keep every 7th block whole
+        L.bits[::7] = 16
+    assert (L.bits == 16).any() and (L.bits != 16).any()
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    check_sched(P, L.bits)
+    for M in (1, 3, 8, 16, 40, 300):
+        x = synth.make_x(9200 + M, M, L.K)
+        y_ref, bnd = oracle.linear(R, x)
+        assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
+
+
+def test_sixteen_bit_range_error(mpq):
+    from block_wise_mixed_b200 import MpqError
+    L = synth.make_layer("r16", 64, 128, 16.0, 9300, "identity", allowed=(16,))
+    W = L.W.copy()
+    W[1, 2] = synth.f32_to_bf16_bits(np.array([1e5], np.float32))[0]
+    with pytest.raises(MpqError) as ei:
+        mpq.pack(dev(W), L.bits)
+    assert ei.value.name == "MPQ_ERR_RANGE"

@@ -12,7 +12,7 @@ from block_wise_mixed_b200 import build, synth
 MAX_UNITS = 148 * 16
 MIN_UNIT_COST = 4096
 WORK = {0: 0, 1: 2048, 2: 2048, 3: 4096, 4: 2304, 5: 4352, 6: 4352, 8: 2560}
-ORDER = [1, 2, 3, 4, 5, 6, 8]
+ORDER = [1, 2, 3, 4, 5, 6, 8, 16]
 DESC = 32
 
 
@@ -23,6 +23,8 @@ def _lib():
 
 
 def block_cost(b):
+    if b == 16:
+        return 16384 + 256 + 272 + 2048
     return 32 if b == 0 else 1024 * b + 256 + 272 + WORK[b]
 
 
@@ -34,7 +36,7 @@ def restated_schedule(N, K, bits):
     NB, KB = N // 64, K // 128
     T = NB * KB
     bits = np.asarray(bits, np.int64)
-    cost = np.array([block_cost(b) if b in WORK else 0 for b in range(9)], np.int64)[bits]
+    cost = np.array([block_cost(b) if (b in WORK or b == 16) else 0 for b in range(17)], np.int64)[bits]
     pre = np.concatenate([[0], np.cumsum(cost)])
     total = int(pre[-1])
     want = max(1, min(-(-total // MIN_UNIT_COST), MAX_UNITS, T))
@@ -62,24 +64,28 @@ def restated_schedule(N, K, bits):
     for b in ORDER:
         seg_off[b] = off
         off += int((bits == b).sum()) * 1024 * b
-    words = DESC * U + 4 * len(nz)
+    nstage = np.where(bits == 16, 2, (bits != 0).astype(np.int64))   # a 16-bit block: two halves
+    words = DESC * U + 4 * int(nstage.sum())
     out = np.zeros(words, np.uint32)
     for u in range(U):
         t0, t1 = bounds[u], bounds[u + 1]
         d = out[DESC * u:DESC * (u + 1)]
         d[0], d[1] = t0, t1
-        d[2] = int((bits[:t0] != 0).sum())
-        d[3] = int((bits[t0:t1] != 0).sum())
+        d[2] = int(nstage[:t0].sum())
+        d[3] = int(nstage[t0:t1].sum())
         ra, rb = t0 // KB, (t1 - 1) // KB
         d[10], d[11], d[12] = row_slot[ra], nc[ra], u - row_first[ra]
         d[13], d[14], d[15] = row_slot[rb], nc[rb], u - row_first[rb]
     st = out[DESC * U:].reshape(-1, 4)
+    si = 0
     for k, t in enumerate(nz):
         b = int(bits[t])
-        st[k, 0] = seg_off[b] + 1024 * b * int((bits[:t] == b).sum())
-        st[k, 1] = 64 * k
-        st[k, 2] = (t % KB) | (b << 16)
-        st[k, 3] = t // KB
+        for half in range(2 if b == 16 else 1):
+            st[si, 0] = seg_off[b] + 1024 * b * int((bits[:t] == b).sum()) + 8192 * half
+            st[si, 1] = 64 * k
+            st[si, 2] = (t % KB) | (b << 16) | (half << 24)
+            st[si, 3] = t // KB
+            si += 1
     return out, bounds, row_slot, nc
 
 
@@ -89,6 +95,7 @@ CASES = [
     ("zero_heavy", synth.make_layer("z", 512, 1024, 0.6, 7, "random")),
     ("one_column", synth.make_layer("c", 1024, 128, 3.0, 8, "identity")),
     ("one_row", synth.make_layer("r", 64, 4096, 2.1, 9, "identity")),
+    ("tilequant_8_16", synth.make_layer("t", 512, 2048, 8.8, 10, "saliency", allowed=(8, 16))),
 ]
 
 
