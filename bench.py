@@ -93,12 +93,12 @@ def load_traffic(kernel: str, workload: str):
 
 def launches_per_call(lay, M, has_row_perm):
     """Kernels one mpq_linear call launches (the library's dispatch rule):
-    M <= 16 -- the activation prologue unless M == 1 on a layer whose runs
+    M <= 8 -- the activation prologue unless M == 1 on a layer whose runs
     hold at most two blocks on average (the decode kernel then builds its own
-    activation records), plus one decode launch per 8 tokens; M > 16 -- the
-    prologue, the tensor-core kernel and, when the rows are reordered, the
-    reordering kernel (split-K partials too)."""
-    if M <= 16:
+    activation records), plus one decode launch; M > 8 -- the prologue, the
+    tensor-core kernel and, when the rows are reordered (or k is split), the
+    reordering kernel."""
+    if M <= 8:
         fused = M == 1 and lay.NB * lay.KB <= 2 * lay.n_units
         return (0 if fused else 1) + (M + 7) // 8
     return 2 + (1 if has_row_perm else 0)

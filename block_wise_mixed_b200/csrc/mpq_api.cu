@@ -26,7 +26,12 @@ namespace {
 constexpr int kMaxUnits = 148 * DEC_CTAS_PER_SM * DEC_WARPS;   // one run per resident decode warp
 constexpr uint64_t kMinUnitCost = 4096; // cost units (bytes) per run, at least
 constexpr int kMaxDecodeTokens = DEC_MAX_TOKENS;   // tokens per decode launch
-constexpr int kDecodeMaxM = 16;         // larger batches take the tensor-core kernel
+// Larger batches take the tensor-core kernel: it streams every weight tile
+// once for any M <= 256 and its time hardly grows with M up to 128, while a
+// decode launch (<= 8 tokens) costs about as much as the whole tensor-core
+// call at M = 8 and twice as much at M = 16 (measured on the 14336 x 4096 and
+// 28672 x 8192 layers).
+constexpr int kDecodeMaxM = 8;
 constexpr int kPackRowsPerCta = 1;
 
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -557,7 +562,7 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
         xc.gridDim = dim3((unsigned)M);
         e = cudaLaunchKernelEx(&xc, k_xprep<XP_PREFILL>, xp);
     } else if (!fused) {
-        const int items = KB * M, per = XPREP_THREADS / 32;
+        const int items = KB * M * 4, per = XPREP_THREADS / 32;   // a warp per digit variant
         xc.gridDim = dim3((unsigned)((items + per - 1) / per));
         e = cudaLaunchKernelEx(&xc, k_xprep_decode, xp);
     } else {

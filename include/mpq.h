@@ -205,10 +205,12 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
  *           cudaMemset); every call that ends without a device error leaves
  *           the parts that must start at zero at zero, so it can be reused
  *           as is (zero it again after a device error).
- * Uses a memory-bound decode kernel for M <= 16 and a tensor-core kernel for
- * larger M.  Non-finite x gives non-finite y (no error).  Activations are
- * moved into fp16 by exact powers of two; for M <= 16 that needs
- * |x| < 2^118 (larger magnitudes overflow to inf).
+ * Uses a memory-bound decode kernel (integer tensor cores) for M <= 8 and a
+ * tcgen05 tensor-core kernel for larger M.  Non-finite x gives non-finite y
+ * (no error).  Activations are scaled by exact powers of two (per 128-column
+ * slice into 23-bit integers for M <= 8, per token into fp16 above); a
+ * slice element more than 2^15 below the slice maximum is rounded to 2^-23
+ * of that maximum.
  * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT. */
 mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M,
                       float* y_dev, void* ws, size_t ws_bytes, void* stream);
