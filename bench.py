@@ -227,7 +227,7 @@ def clone_layer(P):
     from block_wise_mixed_b200 import _lib
     c = {k: (getattr(P, k).clone() if getattr(P, k) is not None else None)
          for k in ("codes", "table", "sched", "scales", "zeros", "row_perm", "col_perm")}
-    layer = _lib.Layer(P.c.N, P.c.K, P.c.n_units, 0, c["codes"].data_ptr(),
+    layer = _lib.Layer(P.c.N, P.c.K, P.c.n_units, P.c.flags, c["codes"].data_ptr(),
                        c["table"].data_ptr(), c["sched"].data_ptr(), c["scales"].data_ptr(),
                        c["zeros"].data_ptr(),
                        c["row_perm"].data_ptr() if c["row_perm"] is not None else None,

@@ -44,7 +44,7 @@ class Layout(ctypes.Structure):
 
 class Layer(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("n_units", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("codes", ctypes.c_void_p),
+                ("flags", ctypes.c_int32), ("codes", ctypes.c_void_p),
                 ("table", ctypes.c_void_p), ("sched", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
                 ("row_perm", ctypes.c_void_p), ("col_perm", ctypes.c_void_p)]
@@ -76,43 +76,59 @@ def load(path: str):
     argument and result types declared."""
     L = ctypes.CDLL(path)
     P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
-    L.mpq_plan.argtypes = [i32, i32, P, ctypes.POINTER(Layout)]
-    L.mpq_plan_schedule.argtypes = [ctypes.POINTER(Layout), P, P]
-    L.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
-    L.mpq_pack_workspace_size.restype = sz
-    L.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
-    L.mpq_pack_timed.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P,
+    class _Decl:
+        """Declares argument/result types of exported functions; a build
+        that lacks one (an older library loaded for comparison) keeps the
+        rest usable, and the missing call fails when used."""
+        def __init__(self, lib):
+            self.lib = lib
+
+        def __getattr__(self, name):
+            f = getattr(self.lib, name, None)
+            return f if f is not None else _Missing()
+
+    class _Missing:
+        def __setattr__(self, k, v):
+            pass
+
+    D = _Decl(L)
+    D.mpq_plan.argtypes = [i32, i32, P, ctypes.POINTER(Layout)]
+    D.mpq_plan_schedule.argtypes = [ctypes.POINTER(Layout), P, P]
+    D.mpq_pack_workspace_size.argtypes = [ctypes.POINTER(Layout)]
+    D.mpq_pack_workspace_size.restype = sz
+    D.mpq_pack.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P]
+    D.mpq_pack_timed.argtypes = [ctypes.POINTER(Layout), P, P, P, P, ctypes.POINTER(Layer), P, sz, P,
                                  P, P]
-    L.mpq_linear_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
-    L.mpq_linear_workspace_size.restype = sz
-    L.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
-    L.mpq_linear_timed.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P, P, P]
-    L.mpq_linear_typed_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_int]
-    L.mpq_linear_typed_workspace_size.restype = sz
-    L.mpq_linear_typed.argtypes = [ctypes.POINTER(Layer), P, i32, P, ctypes.c_int, P, sz, P]
-    L.mpq_linear_group_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, i32]
-    L.mpq_linear_group_workspace_size.restype = sz
-    L.mpq_linear_group.argtypes = [ctypes.POINTER(Layer), i32, P, i32, P, P, sz, P]
-    L.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
-    L.mpq_linear_host_workspace_size.restype = sz
-    L.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
-    L.mpq_linear_noalloc.argtypes = [ctypes.POINTER(Layer), P, i32, P, P]
-    L.mpq_linear_noalloc.restype = ctypes.c_int
-    L.mpq_noalloc_check.argtypes = [P]
-    L.mpq_noalloc_check.restype = ctypes.c_int
-    L.mpq_allocate_bits_workspace_size.argtypes = [ctypes.c_int64]
-    L.mpq_allocate_bits_workspace_size.restype = sz
-    L.mpq_allocate_bits.argtypes = [ctypes.c_int64, P, ctypes.c_uint32, ctypes.c_uint64, P, P, P, sz, P]
-    L.mpq_allocate_bits.restype = ctypes.c_int
-    L.mpq_fold_orders.argtypes = [i32, P, P, P]
-    L.mpq_fold_orders.restype = ctypes.c_int
-    L.mpq_check.argtypes = [P, P]
-    L.mpq_status_string.argtypes = [ctypes.c_int]
-    L.mpq_status_string.restype = ctypes.c_char_p
+    D.mpq_linear_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
+    D.mpq_linear_workspace_size.restype = sz
+    D.mpq_linear.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
+    D.mpq_linear_timed.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P, P, P]
+    D.mpq_linear_typed_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, ctypes.c_int]
+    D.mpq_linear_typed_workspace_size.restype = sz
+    D.mpq_linear_typed.argtypes = [ctypes.POINTER(Layer), P, i32, P, ctypes.c_int, P, sz, P]
+    D.mpq_linear_group_workspace_size.argtypes = [ctypes.POINTER(Layer), i32, i32]
+    D.mpq_linear_group_workspace_size.restype = sz
+    D.mpq_linear_group.argtypes = [ctypes.POINTER(Layer), i32, P, i32, P, P, sz, P]
+    D.mpq_linear_host_workspace_size.argtypes = [ctypes.POINTER(Layer), i32]
+    D.mpq_linear_host_workspace_size.restype = sz
+    D.mpq_linear_host.argtypes = [ctypes.POINTER(Layer), P, i32, P, P, sz, P]
+    D.mpq_linear_noalloc.argtypes = [ctypes.POINTER(Layer), P, i32, P, P]
+    D.mpq_linear_noalloc.restype = ctypes.c_int
+    D.mpq_noalloc_check.argtypes = [P]
+    D.mpq_noalloc_check.restype = ctypes.c_int
+    D.mpq_allocate_bits_workspace_size.argtypes = [ctypes.c_int64]
+    D.mpq_allocate_bits_workspace_size.restype = sz
+    D.mpq_allocate_bits.argtypes = [ctypes.c_int64, P, ctypes.c_uint32, ctypes.c_uint64, P, P, P, sz, P]
+    D.mpq_allocate_bits.restype = ctypes.c_int
+    D.mpq_fold_orders.argtypes = [i32, P, P, P]
+    D.mpq_fold_orders.restype = ctypes.c_int
+    D.mpq_check.argtypes = [P, P]
+    D.mpq_status_string.argtypes = [ctypes.c_int]
+    D.mpq_status_string.restype = ctypes.c_char_p
     for f in ("mpq_plan", "mpq_pack", "mpq_pack_timed", "mpq_linear", "mpq_linear_typed",
               "mpq_linear_group", "mpq_linear_timed", "mpq_linear_host",
               "mpq_check"):
-        getattr(L, f).restype = ctypes.c_int
+        getattr(D, f).restype = ctypes.c_int
     return L
 
 
@@ -188,7 +204,8 @@ def alloc_layer(L: Layout, device, has_row_perm: bool, has_col_perm: bool) -> Pa
     zeros = buf(2 * L.n_sz)
     rp = torch.empty(L.N, dtype=torch.int32, device=device) if has_row_perm else None
     cp = torch.empty(L.K, dtype=torch.int32, device=device) if has_col_perm else None
-    c = Layer(L.N, L.K, L.n_units, 0, codes.data_ptr(), table.data_ptr(), sched.data_ptr(),
+    c = Layer(L.N, L.K, L.n_units, LAYER_16BIT if L.seg_bytes[16] else 0, codes.data_ptr(),
+              table.data_ptr(), sched.data_ptr(),
               scales.data_ptr(), zeros.data_ptr(),
               rp.data_ptr() if rp is not None else None,
               cp.data_ptr() if cp is not None else None)
@@ -229,6 +246,7 @@ def linear_workspace_size(layer: PackedLayer, M: int) -> int:
 
 
 Y_F32, Y_BF16 = 0, 1   # mpq_ydtype
+LAYER_16BIT = 1        # mpq_layer.flags: the layer has 16-bit blocks
 
 
 def linear_typed_workspace_size(layer: PackedLayer, M: int, ydtype: int = Y_F32) -> int:
@@ -362,7 +380,7 @@ def with_orders(P: PackedLayer, row_perm=None, col_perm=None, keep_rows=True, ke
     orders (device int32 tensors or None): the packed buffers are shared."""
     rp = P.row_perm if keep_rows else row_perm
     cp = P.col_perm if keep_cols else col_perm
-    c = Layer(P.c.N, P.c.K, P.c.n_units, 0, P.c.codes, P.c.table, P.c.sched, P.c.scales, P.c.zeros,
+    c = Layer(P.c.N, P.c.K, P.c.n_units, P.c.flags, P.c.codes, P.c.table, P.c.sched, P.c.scales, P.c.zeros,
               rp.data_ptr() if rp is not None else None, cp.data_ptr() if cp is not None else None)
     return PackedLayer(P.layout, P.codes, P.table, P.sched, P.scales, P.zeros, rp, cp, c)
 

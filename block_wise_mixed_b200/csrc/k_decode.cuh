@@ -353,11 +353,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 // holds columns 32t + 4ks .. +3, so each lane reads 64 contiguous bytes of a
 // row and of the activation slice (the bf16 variant is x' in column order).
 // mma rows: tile tt, row g = half row 16tt + g, row g + 8 = 16tt + g + 8;
-// columns = tokens 0..7.  The results go through the stage's fix-up area to
-// the lanes that own the rows in the quantized path (rows 8g + 2i + (t & 1)).
-template <int G>
-__device__ __forceinline__ void block_accumulate16(const uint8_t* stage, const uint8_t* xb, float* fix,
-                                                   int half, int g, int t, uint32_t Mg, float (&acc)[4][G]) {
+// columns = tokens 0..7.  The sums go to the stage's fix-up area
+// (fix[half row][token]); block_add16 hands them to the lanes that own the
+// rows in the quantized path.  Kept out of line: 16-bit blocks are few, and
+// the hot loop's code stays small.
+__device__ __noinline__ void block_mma16(const uint8_t* stage, const uint8_t* xb, float* fix, int g, int t,
+                                         uint32_t Mg) {
     uint32_t b[16];
     {
         const uint8_t* src = (uint32_t)g < Mg ? xb + g * XQD_VAR + 64 * t : nullptr;
@@ -392,15 +393,21 @@ __device__ __forceinline__ void block_accumulate16(const uint8_t* stage, const u
         if (t1 < Mg) { fix[ra * Mg + t1] = c[1] + d[1]; fix[rb * Mg + t1] = c[3] + d[3]; }
     }
     __syncwarp();
-    if ((g >> 2) == half) {   // this lane's rows 8g + 2i + (t & 1) lie in the half
+}
+
+// The owners of the half's rows add the fix-up area's sums (rows 8g + 2i +
+// (t & 1) lie in half `half` when g / 4 == half).
+template <int G>
+__device__ __forceinline__ void block_add16(const float* fix, int half, int g, int t, uint32_t Mg,
+                                            float (&acc)[4][G]) {
+    if ((g >> 2) != half) return;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int rl = 8 * g + 2 * i + (t & 1) - 32 * half;
+    for (int i = 0; i < 4; ++i) {
+        const int rl = 8 * g + 2 * i + (t & 1) - 32 * half;
 #pragma unroll
-            for (int grp = 0; grp < G; ++grp) {
-                const uint32_t tok = 2u * grp + (uint32_t)(t >> 1);
-                if (tok < Mg) acc[i][grp] += fix[rl * Mg + tok];
-            }
+        for (int grp = 0; grp < G; ++grp) {
+            const uint32_t tok = 2u * grp + (uint32_t)(t >> 1);
+            if (tok < Mg) acc[i][grp] += fix[rl * Mg + tok];
         }
     }
 }
@@ -479,6 +486,7 @@ __device__ __forceinline__ int4 fused_cols(const DecodeParams& p, uint32_t kb, i
     return __ldg(reinterpret_cast<const int4*>(p.col_perm + c0));
 }
 
+template <bool W16>
 __device__ __forceinline__ void fused_records(const DecodeParams& p, int4 cp, int b, uint8_t* rec, int lane) {
     const uint16_t* xr = p.x + (size_t)p.m0 * p.K;
     float v[4];
@@ -486,7 +494,7 @@ __device__ __forceinline__ void fused_records(const DecodeParams& p, int4 cp, in
     v[1] = __uint_as_float((uint32_t)xr[cp.y] << 16);
     v[2] = __uint_as_float((uint32_t)xr[cp.z] << 16);
     v[3] = __uint_as_float((uint32_t)xr[cp.w] << 16);
-    if (b == 16) {   // the bf16 slice, column order
+    if (W16 && b == 16) {   // the bf16 slice, column order
         *reinterpret_cast<uint2*>(rec + 8 * lane) =
             make_uint2((uint32_t)xr[cp.x] | ((uint32_t)xr[cp.y] << 16), (uint32_t)xr[cp.z] | ((uint32_t)xr[cp.w] << 16));
         fence_proxy_async_smem();
@@ -507,7 +515,7 @@ __device__ __forceinline__ void fused_records(const DecodeParams& p, int4 cp, in
 // One warp's run u of the layer p (the body of the decode kernels below).
 // G token groups of two: the launch's tokens Mg <= 2G.
 // ---------------------------------------------------------------------------
-template <int G, bool FUSED_X>
+template <int G, bool FUSED_X, bool W16>
 __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, int u, int lane) {
     const int g = lane >> 2, t = lane & 3;
     const uint32_t KB = (uint32_t)p.KB;
@@ -560,21 +568,28 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
     auto issue_more = [&]() {
         while (q_tail - q_head < (uint32_t)DEC_SLOTS && next < ns && !aborted && !(kWaitTest && q_tail > 0)) {
             const int l = (int)(next & 31u);
-            const uint32_t coff = __shfl_sync(0xffffffffu, cs.x, l);
-            const uint32_t szo = __shfl_sync(0xffffffffu, cs.y, l);
+            // the stage's size first: when the ring is full nothing else is needed
             const uint32_t kbb = __shfl_sync(0xffffffffu, cs.z, l);
-            const uint32_t nbs = __shfl_sync(0xffffffffu, cs.w, l);
             const uint32_t b = (kbb >> 16) & 0xFFu;
-            const uint32_t hb = kbb >> 24;                 // 16-bit blocks: which row half
-            const uint32_t xo = (kbb & 0xFFFFu) * rec_bytes + var_lo(b) * var_bytes + x_tok_off;
+            if (!W16 && b == 16u) {   // a 16-bit block in a layer not flagged for them
+                if (lane == 0) set_error(p.err, MPQ_ERR_BITS);
+                aborted = true;
+                break;
+            }
+            const bool b16 = W16 && b == 16u;
             const uint32_t xb = split_width((int)b) ? 2u * x_bytes : x_bytes;
-            const uint32_t pay = b == 16 ? 8192u : 1024u * b + 256u;   // payload (+ scales, zeros)
-            const uint32_t size = pay + xb + (b == 16 ? 128u * Mg : 0u);   // stage_bytes(b, Mg)
+            const uint32_t pay = b16 ? 8192u : 1024u * b + 256u;   // payload (+ scales, zeros)
+            const uint32_t size = pay + xb + (b16 ? 128u * Mg : 0u);   // stage_bytes(b, Mg)
             if (q_head == q_tail) { r_head = 0; r_tail = 0; r_pos = 0; }   // empty ring: restart at 0
             // a stage never wraps: when the ring's tail end is too short, skip to 0
             const bool skip = r_pos + size > (uint32_t)DEC_RING;
             const uint32_t start = skip ? r_head + ((uint32_t)DEC_RING - r_pos) : r_head;
             if (start + size - r_tail > (uint32_t)DEC_RING) break;   // ring full: compute first
+            const uint32_t coff = __shfl_sync(0xffffffffu, cs.x, l);
+            const uint32_t szo = __shfl_sync(0xffffffffu, cs.y, l);
+            const uint32_t nbs = __shfl_sync(0xffffffffu, cs.w, l);
+            const uint32_t hb = kbb >> 24;                 // 16-bit blocks: which row half
+            const uint32_t xo = (kbb & 0xFFFFu) * rec_bytes + var_lo(b) * var_bytes + x_tok_off;
             const uint32_t slot = q_tail % DEC_SLOTS;
             const uint32_t off = skip ? 0u : r_pos;
             if (lane == 0) {
@@ -584,7 +599,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
                 mbar_arrive_expect_tx(bar, FUSED_X ? pay : pay + xb);
                 uint8_t* dst = W.ring + off;
                 if (!kWaitTest) {
-                    if (b == 16) {
+                    if (b16) {
                         bulk_g2s(dst, p.codes + coff, 8192u, bar);
                     } else {
                         bulk_g2s(dst, p.codes + coff, 1024u * b, bar);
@@ -625,7 +640,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             const uint32_t kbits = __shfl_sync(0xffffffffu, qe_bits, slot) & 0xFFu;
             const uint32_t ko = __shfl_sync(0xffffffffu, qe_off, slot);
             const uint32_t kx = __shfl_sync(0xffffffffu, qe_x, slot);
-            const uint32_t kpay = kbits == 16 ? 8192u : 1024u * kbits + 256u;
+            const uint32_t kpay = (W16 && kbits == 16) ? 8192u : 1024u * kbits + 256u;
             if (lane == 0 && !kWaitTest) issue_x(W.ring + ko + kpay, kbits, kx, &W.full[slot]);
         }
     }
@@ -666,18 +681,19 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             }
             if (!aborted) {
                 const uint8_t* stage = W.ring + foff;
-                uint8_t* xs = W.ring + foff + (fb == 16 ? 8192u : 1024u * fb + 256u);
+                uint8_t* xs = W.ring + foff + ((W16 && fb == 16) ? 8192u : 1024u * fb + 256u);
                 if (FUSED_X) {
                     const uint32_t kb = __shfl_sync(0xffffffffu, qe_kb, slot);
                     const int4 cp = (kb == cp_kb) ? cp_pref : fused_cols(p, kb, lane);
-                    fused_records(p, cp, (int)fb, xs, lane);
+                    fused_records<W16>(p, cp, (int)fb, xs, lane);
                 }
                 const uint8_t* xh = xs + x_bytes;
                 const uint8_t* z32 = reinterpret_cast<const uint8_t*>(W.zero32);
-                if (fb == 16)
-                    block_accumulate16<G>(stage, xs, reinterpret_cast<float*>(xs + x_bytes), (int)(fbh >> 8), g, t,
-                                          Mg, acc);
-                else switch (fb) {
+                if (W16 && fb == 16) {
+                    float* fix = reinterpret_cast<float*>(xs + x_bytes);
+                    block_mma16(stage, xs, fix, g, t, Mg);
+                    block_add16<G>(fix, (int)(fbh >> 8), g, t, Mg, acc);
+                } else switch (fb) {
                     case 1: block_accumulate<1, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
                     case 2: block_accumulate<2, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
                     case 3: block_accumulate<3, G>(stage, xs, xh, z32, g, t, Mg, acc); break;
@@ -773,12 +789,14 @@ __device__ __forceinline__ DecWarp& decode_prologue(uint8_t* smem_raw, int warp,
 template <int G>
 struct DecRegs { static constexpr int value = G == 1 ? DEC_MAX_REGS : 168; };
 
-template <int G, bool FUSED_X = false>
+// W16: built with the 16-bit passthrough path (for layers flagged to have
+// 16-bit blocks; the others take the smaller code).
+template <int G, bool FUSED_X = false, bool W16 = false>
 __global__ void __maxnreg__(DecRegs<G>::value) k_decode(DecodeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     DecWarp& W = decode_prologue(smem_raw, warp, lane);
-    decode_warp<G, FUSED_X>(p, W, (int)blockIdx.x * DEC_WARPS + warp, lane);
+    decode_warp<G, FUSED_X, W16>(p, W, (int)blockIdx.x * DEC_WARPS + warp, lane);
 }
 
 // Several layers that share x in one launch (one token, fused activation
@@ -790,6 +808,7 @@ struct DecodeGroup {
     int n;
 };
 
+template <bool W16 = false>
 __global__ void __maxnreg__(DEC_MAX_REGS) k_decode_group(const __grid_constant__ DecodeGroup gp) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -798,7 +817,7 @@ __global__ void __maxnreg__(DEC_MAX_REGS) k_decode_group(const __grid_constant__
     if (v >= gp.unit_begin[gp.n]) return;
     int l = 0;
     while (l + 1 < gp.n && v >= gp.unit_begin[l + 1]) ++l;
-    decode_warp<1, true>(gp.layer[l], W, v - gp.unit_begin[l], lane);
+    decode_warp<1, true, W16>(gp.layer[l], W, v - gp.unit_begin[l], lane);
 }
 
 }  // namespace mpq

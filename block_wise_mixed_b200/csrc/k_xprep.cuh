@@ -235,16 +235,16 @@ constexpr int XPREP_DEC_WARPS = XPREP_THREADS / 32;
 
 __global__ void __launch_bounds__(XPREP_THREADS, 8) k_xprep_decode(XprepParams p) {
     pdl_launch_dependents();
+    // one variant at a time per warp (small, so that the CTAs fit beside the
+    // decode kernel's on an SM; few CTAs, so that they keep few SMs from
+    // taking the next decode launch's CTAs while they wait for the kernel
+    // before)
     __shared__ __align__(16) uint8_t recs[XPREP_DEC_WARPS][XQD_VAR];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int KB = p.K / 128;
-    // one warp per (block column, token, digit variant): the four variants of
-    // a slice are built side by side (the slice's integers are recomputed by
-    // each; the warp of variant 3 also writes the bf16 variant)
-    const int item = blockIdx.x * XPREP_DEC_WARPS + warp;   // = (kb * M + m) * 4 + vv
-    const bool active = item < KB * p.M * 4;
-    const int vv = item & 3, km = item >> 2;
-    const int kb = active ? km / p.M : 0, m = active ? km % p.M : 0;
+    const int item = blockIdx.x * XPREP_DEC_WARPS + warp;   // = kb * M + m
+    const bool active = item < KB * p.M;
+    const int kb = active ? item / p.M : 0, m = active ? item % p.M : 0;
     // lane holds columns 4*lane .. 4*lane+3 of the slice; the column order is
     // static, so it is read before waiting for the kernel that writes x
     const int c0 = kb * 128 + 4 * lane;
@@ -266,14 +266,20 @@ __global__ void __launch_bounds__(XPREP_THREADS, 8) k_xprep_decode(XprepParams p
     float F;
     xqd_integerize(v, X, T, F);
     uint8_t* rs = recs[warp];
+    // variant vv of token m of block column kb
     uint8_t* rec = reinterpret_cast<uint8_t*>(p.xq) + (size_t)kb * p.M * XQD_REC + (size_t)m * XQD_VAR;
-    xqd_scatter_variant(X, T, F, vv, rs, lane);
-    __syncwarp();
-    if (lane < XQD_VAR / 16)
-        reinterpret_cast<uint4*>(rec + (size_t)vv * p.M * XQD_VAR)[lane] = reinterpret_cast<const uint4*>(rs)[lane];
-    if (vv == 3)   // variant 4: the bf16 slice in column order
-        *reinterpret_cast<uint2*>(rec + (size_t)4 * p.M * XQD_VAR + 8 * lane) =
-            make_uint2((uint32_t)xr[cp.x] | ((uint32_t)xr[cp.y] << 16), (uint32_t)xr[cp.z] | ((uint32_t)xr[cp.w] << 16));
+#pragma unroll 1
+    for (int vv = 0; vv < 4; ++vv) {
+        xqd_scatter_variant(X, T, F, vv, rs, lane);
+        __syncwarp();
+        if (lane < XQD_VAR / 16)
+            reinterpret_cast<uint4*>(rec + (size_t)vv * p.M * XQD_VAR)[lane] =
+                reinterpret_cast<const uint4*>(rs)[lane];
+        __syncwarp();
+    }
+    // variant 4: the bf16 slice in column order
+    *reinterpret_cast<uint2*>(rec + (size_t)4 * p.M * XQD_VAR + 8 * lane) =
+        make_uint2((uint32_t)xr[cp.x] | ((uint32_t)xr[cp.y] << 16), (uint32_t)xr[cp.z] | ((uint32_t)xr[cp.w] << 16));
 }
 
 }  // namespace mpq

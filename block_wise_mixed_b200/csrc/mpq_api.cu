@@ -301,6 +301,11 @@ cudaError_t ensure_smem_attr(F* kernel, int bytes, std::atomic<uint64_t>& done) 
 std::atomic<uint64_t> g_decode_attr{0};
 std::atomic<uint64_t> g_decode_attr8{0};
 std::atomic<uint64_t> g_decode_attr16{0};
+std::atomic<uint64_t> g_decode_attr_w{0};
+std::atomic<uint64_t> g_decode_attr8_w{0};
+std::atomic<uint64_t> g_decode_attr16_w{0};
+std::atomic<uint64_t> g_decode_attr_f_w{0};
+std::atomic<uint64_t> g_decode_attr_g_w{0};
 std::atomic<uint64_t> g_decode_attr_f{0};
 std::atomic<uint64_t> g_decode_attr_g{0};
 std::atomic<uint64_t> g_prefill_attr{0};
@@ -562,7 +567,7 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
         xc.gridDim = dim3((unsigned)M);
         e = cudaLaunchKernelEx(&xc, k_xprep<XP_PREFILL>, xp);
     } else if (!fused) {
-        const int items = KB * M * 4, per = XPREP_THREADS / 32;   // a warp per digit variant
+        const int items = KB * M, per = XPREP_THREADS / 32;
         xc.gridDim = dim3((unsigned)((items + per - 1) / per));
         e = cudaLaunchKernelEx(&xc, k_xprep_decode, xp);
     } else {
@@ -641,10 +646,18 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
         return MPQ_OK;
     }
 
-    e = ensure_smem_attr(k_decode<1>, (int)sizeof(DecSmem), g_decode_attr);
-    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<2>, (int)sizeof(DecSmem), g_decode_attr8);
-    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<4>, (int)sizeof(DecSmem), g_decode_attr16);
-    if (e == cudaSuccess) e = ensure_smem_attr(k_decode<1, true>, (int)sizeof(DecSmem), g_decode_attr_f);
+    const bool w16 = (layer->flags & MPQ_LAYER_16BIT) != 0;
+    e = w16 ? ensure_smem_attr(k_decode<1, false, true>, (int)sizeof(DecSmem), g_decode_attr_w)
+            : ensure_smem_attr(k_decode<1>, (int)sizeof(DecSmem), g_decode_attr);
+    if (e == cudaSuccess)
+        e = w16 ? ensure_smem_attr(k_decode<2, false, true>, (int)sizeof(DecSmem), g_decode_attr8_w)
+                : ensure_smem_attr(k_decode<2>, (int)sizeof(DecSmem), g_decode_attr8);
+    if (e == cudaSuccess)
+        e = w16 ? ensure_smem_attr(k_decode<4, false, true>, (int)sizeof(DecSmem), g_decode_attr16_w)
+                : ensure_smem_attr(k_decode<4>, (int)sizeof(DecSmem), g_decode_attr16);
+    if (e == cudaSuccess)
+        e = w16 ? ensure_smem_attr(k_decode<1, true, true>, (int)sizeof(DecSmem), g_decode_attr_f_w)
+                : ensure_smem_attr(k_decode<1, true>, (int)sizeof(DecSmem), g_decode_attr_f);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
     DecodeParams dp = decode_params(layer, x_dev, M, y_dev, w);
 
@@ -664,10 +677,16 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
         dp.m0 = m0;
         dp.Mg = std::min(kMaxDecodeTokens, M - m0);
         // token groups of two: one for up to 2 tokens, two for 4, four for 8
-        e = fused ? cudaLaunchKernelEx(&cfg, k_decode<1, true>, dp)
-            : dp.Mg <= 2 ? cudaLaunchKernelEx(&cfg, k_decode<1>, dp)
-            : dp.Mg <= 4 ? cudaLaunchKernelEx(&cfg, k_decode<2>, dp)
-                         : cudaLaunchKernelEx(&cfg, k_decode<4>, dp);
+        if (w16)
+            e = fused ? cudaLaunchKernelEx(&cfg, k_decode<1, true, true>, dp)
+                : dp.Mg <= 2 ? cudaLaunchKernelEx(&cfg, k_decode<1, false, true>, dp)
+                : dp.Mg <= 4 ? cudaLaunchKernelEx(&cfg, k_decode<2, false, true>, dp)
+                             : cudaLaunchKernelEx(&cfg, k_decode<4, false, true>, dp);
+        else
+            e = fused ? cudaLaunchKernelEx(&cfg, k_decode<1, true>, dp)
+                : dp.Mg <= 2 ? cudaLaunchKernelEx(&cfg, k_decode<1>, dp)
+                : dp.Mg <= 4 ? cudaLaunchKernelEx(&cfg, k_decode<2>, dp)
+                             : cudaLaunchKernelEx(&cfg, k_decode<4>, dp);
         if (e != cudaSuccess) return MPQ_ERR_CUDA;
     }
     if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess)
@@ -734,7 +753,10 @@ mpq_status mpq_linear_group(const mpq_layer* layers, int32_t n, const void* x_de
         return MPQ_OK;
     }
     // one launch over all the layers' runs
-    cudaError_t e = ensure_smem_attr(k_decode_group, (int)sizeof(DecSmem), g_decode_attr_g);
+    bool w16 = false;
+    for (int i = 0; i < n; ++i) w16 = w16 || (layers[i].flags & MPQ_LAYER_16BIT) != 0;
+    cudaError_t e = w16 ? ensure_smem_attr(k_decode_group<true>, (int)sizeof(DecSmem), g_decode_attr_g_w)
+                        : ensure_smem_attr(k_decode_group<false>, (int)sizeof(DecSmem), g_decode_attr_g);
     if (e != cudaSuccess) return MPQ_ERR_CUDA;
     DecodeGroup gp{};
     gp.n = n;
@@ -753,7 +775,8 @@ mpq_status mpq_linear_group(const mpq_layer* layers, int32_t n, const void* x_de
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, k_decode_group, gp));
+    return cuda_status(w16 ? cudaLaunchKernelEx(&cfg, k_decode_group<true>, gp)
+                           : cudaLaunchKernelEx(&cfg, k_decode_group<false>, gp));
 }
 
 size_t mpq_linear_host_workspace_size(const mpq_layer* layer, int32_t M) {

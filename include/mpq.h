@@ -131,10 +131,17 @@ typedef struct {
 
 /* A packed layer: device pointers to caller-owned buffers of the sizes in
  * mpq_layout.  mpq_pack writes these buffers; mpq_linear reads them. */
+/* mpq_layer.flags */
+#define MPQ_LAYER_16BIT 1   /* the layer has 16-bit blocks (seg_bytes[16] > 0) */
+
 typedef struct {
     int32_t N, K;
     int32_t n_units;
-    int32_t reserved;
+    int32_t flags;               /* MPQ_LAYER_16BIT when the layer has 16-bit
+                                    blocks: mpq_linear then uses the decode
+                                    kernel built with the 16-bit path (a 16-bit
+                                    block met without the flag records
+                                    MPQ_ERR_BITS on the device)                */
     const void* codes;           /* uint8  [codes_bytes]                        */
     const mpq_block* table;      /* [NB*KB]                                      */
     const uint32_t* sched;       /* [sched_words] (mpq_layout)                    */
@@ -211,7 +218,8 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
  * slice into 23-bit integers for M <= 8, per token into fp16 above); a
  * slice element more than 2^15 below the slice maximum is rounded to 2^-23
  * of that maximum.
- * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT. */
+ * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT, BITS (a
+ * 16-bit block in a layer whose flags lack MPQ_LAYER_16BIT). */
 mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M,
                       float* y_dev, void* ws, size_t ws_bytes, void* stream);
 
