@@ -1,5 +1,5 @@
 """block_wise_mixed_b200 -- block-wise mixed-precision weight-only quantized
-linear layer (64x128 blocks, per-block bits in {0,1,2,3,4,5,6,8}, RTN-g128,
+linear layer (64x128 blocks, per-block bits in {0,1,2,3,4,5,6,8} plus 16-bit passthrough blocks, RTN-g128,
 fp16 scale/zero, bi-directional channel reordering) on NVIDIA B200.
 
 The computation lives in the C-ABI library ``libmpq.so`` (include/mpq.h); this

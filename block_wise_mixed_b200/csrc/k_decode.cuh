@@ -573,7 +573,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
             const uint32_t b = (kbb >> 16) & 0xFFu;
             if (!W16 && b == 16u) {   // a 16-bit block in a layer not flagged for them
                 if (lane == 0) set_error(p.err, MPQ_ERR_BITS);
-                aborted = true;
+                next = ns;   // issue nothing more; the stages in flight are consumed as usual
                 break;
             }
             const bool b16 = W16 && b == 16u;
@@ -758,6 +758,11 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& p, DecWarp& W, i
                           p.N, W.rows, lane);
         if (lane == 0) p.counters[nb] = 0u;   // ready for the next launch
     }
+    // after a wait ran out, copies may still be landing in this warp's ring:
+    // wait (bounded) for the last stage issued on each slot before leaving
+    if (aborted && lane == 0)
+        for (uint32_t k = q_tail > (uint32_t)DEC_SLOTS ? q_tail - DEC_SLOTS : 0u; k < q_tail; ++k)
+            mbar_wait_bounded(&W.full[k % DEC_SLOTS], (k / DEC_SLOTS) & 1u, DEC_WAIT_NS);
 }
 
 

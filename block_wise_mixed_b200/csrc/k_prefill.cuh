@@ -362,6 +362,8 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
     };
     auto bits_of = [&](int h, int kb) -> uint32_t { return tbits[h * KB + kb]; };
 
+    // stages armed by the two copy producers (lane 0), for the drain after an abort
+    int c_armed = 0, b_armed = 0;
     if (warp == 0) {
         // -------------------- producer of the packed codes --------------------
         // runs as far ahead as the code stages allow (the weights do not
@@ -400,6 +402,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                         // uses, come before this use's bulk copies
                         fence_proxy_async_smem();
                         mbar_arrive_expect_tx(&S.full_c[sc], bytes);
+                        c_armed = a + 1;
                         if (kWaitTest) {
                             // wait-test build: armed, no copy; the consumers' waits run out
                         } else if (q0) {
@@ -433,6 +436,7 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                     const uint32_t ps = (uint32_t)(bq / PF_B_STAGES) & 1u;
                     if (!mbar_wait_bounded(&S.empty_b[s], ps ^ 1u, DEC_WAIT_NS)) { timed_out(); break; }
                     mbar_arrive_expect_tx(&S.full_b[s], (uint32_t)Cfg::B_BYTES);
+                    b_armed = bq + 1;
                     tma_load_2d(S.b[s], &tmap_x, (kb0 + kb) * 128 + 64 * hh, m0, &S.full_b[s]);
                 }
             }
@@ -560,6 +564,20 @@ k_prefill(PrefillParams p, const __grid_constant__ CUtensorMap tmap_x) {
                 }
             }
         }
+    }
+    // after an abort, copies and tensor-core work may still be in flight into
+    // this CTA's shared memory and TMEM: wait for them (bounded) before the
+    // TMEM is freed and the CTA leaves.  A stage's last arm is the only one
+    // that can be pending (a stage is re-armed only after it was consumed).
+    __syncthreads();
+    if (S.abort_flag && lane == 0) {
+        if (warp == 0)
+            for (int i = max(0, c_armed - PF_C_STAGES); i < c_armed; ++i)
+                mbar_wait_bounded(&S.full_c[i % PF_C_STAGES], (uint32_t)(i / PF_C_STAGES) & 1u, DEC_WAIT_NS);
+        if (warp == PF_WARPS - 1)
+            for (int i = max(0, b_armed - PF_B_STAGES); i < b_armed; ++i)
+                mbar_wait_bounded(&S.full_b[i % PF_B_STAGES], (uint32_t)(i / PF_B_STAGES) & 1u, DEC_WAIT_NS);
+        if (warp == 1) mbar_wait_bounded(&S.d_full, 0u, DEC_WAIT_NS);   // all issued MMAs
     }
     tc_fence_before();
     __syncthreads();

@@ -41,8 +41,10 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
     pdl_launch_dependents();
     pdl_wait();
     __shared__ float red[XPREP_THREADS / 32];
+    // CTA (m, y) converts the y-th of gridDim.y column ranges of token m
+    // (every CTA of the token finds the row maximum itself)
     const int m = blockIdx.x, tid = threadIdx.x, K = p.K;
-    if (m == 0) {
+    if (m == 0 && blockIdx.y == 0) {
         if (p.counters)
             for (int i = tid; i < p.n_counters; i += XPREP_THREADS) p.counters[i] = 0u;
     }
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
     amax = red[0];
     int e = 0;
     if (amax > 0.f && isfinite(amax)) e = min(max(14 - ilogbf(amax), -126), 126);
-    if (tid == 0) p.tok_scale[m] = ldexpf(1.f, -e);
+    if (tid == 0 && blockIdx.y == 0) p.tok_scale[m] = ldexpf(1.f, -e);
 
     auto load = [&](int j) -> float {
         int c = p.col_perm ? p.col_perm[j] : j;
@@ -86,7 +88,9 @@ __global__ void __launch_bounds__(XPREP_THREADS) k_xprep(XprepParams p) {
     };
     {
         __half2* out = reinterpret_cast<__half2*>(p.xq + (size_t)m * K);
-        for (int c2 = tid; c2 < K / 2; c2 += XPREP_THREADS) {
+        const int per = (K / 2 + gridDim.y - 1) / gridDim.y;
+        const int c_end = min(K / 2, ((int)blockIdx.y + 1) * per);
+        for (int c2 = (int)blockIdx.y * per + tid; c2 < c_end; c2 += XPREP_THREADS) {
             const int kb = c2 >> 6, r = c2 & 63, i = r >> 2, j = r & 3;
             const int col = kb * 128 + 8 * i + j;
             out[c2] = __halves2half2(__float2half_rn(load(col)), __float2half_rn(load(col + 4)));

@@ -564,7 +564,9 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
     cudaError_t e;
     if (use_tc) {
         xp.counters = nullptr;
-        xc.gridDim = dim3((unsigned)M);
+        // few tokens: several CTAs per token, about two waves in all
+        const int per_token = std::max(1, std::min(layer->K / 1024, (2 * 148 + M - 1) / M));
+        xc.gridDim = dim3((unsigned)M, (unsigned)per_token);
         e = cudaLaunchKernelEx(&xc, k_xprep<XP_PREFILL>, xp);
     } else if (!fused) {
         const int items = KB * M, per = XPREP_THREADS / 32;

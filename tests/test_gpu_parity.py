@@ -444,3 +444,32 @@ def test_sixteen_bit_range_error(mpq):
     with pytest.raises(MpqError) as ei:
         mpq.pack(dev(W), L.bits)
     assert ei.value.name == "MPQ_ERR_RANGE"
+
+
+@pytest.mark.parametrize("M", [1, 3])     # fused one-token decode; decode after the prologue
+def test_sixteen_bit_block_without_flag(mpq, oracle, M):
+    """A layer whose 16-bit blocks are not announced in mpq_layer.flags runs
+    the decode kernel built without the 16-bit path: the device reports
+    MPQ_ERR_BITS (through mpq_check) instead of computing them, and the
+    context stays usable (the flagged layer then matches the oracle)."""
+    import ctypes
+    import torch
+    from block_wise_mixed_b200 import MpqError, _lib
+    L = synth.make_layer("nf", 256, 1024, 4.0, 9400, "random", allowed=(2, 4, 16))
+    L.bits[::5] = 16
+    P = pack_gpu(mpq, L)
+    assert P.c.flags == _lib.LAYER_16BIT
+    c = _lib.Layer.from_buffer_copy(P.c)
+    c.flags = 0
+    x = dev(synth.make_x(9401 + M, M, L.K))
+    y = torch.empty((M, L.N), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(mpq.linear_workspace_size(P, M), dtype=torch.uint8, device="cuda")
+    st = _lib.lib().mpq_linear(ctypes.byref(c), x.data_ptr(), M, y.data_ptr(), ws.data_ptr(), ws.numel(),
+                               _lib._stream(None))
+    assert st == 0
+    with pytest.raises(MpqError) as ei:
+        _lib.check(ws)
+    assert ei.value.name == "MPQ_ERR_BITS"
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    y_ref, bnd = oracle.linear(R, synth.make_x(9401 + M, M, L.K))
+    assert_y_close(run_linear(mpq, P, synth.make_x(9401 + M, M, L.K)), y_ref, bnd)
