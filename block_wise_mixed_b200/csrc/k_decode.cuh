@@ -20,16 +20,20 @@
 // one it computes.
 //
 // Arithmetic (exact up to the final fp32 steps).  The activation slice is
-// held as integers X (k_xprep.cuh: X = rne(x' 2^e), |X| < 2^15, two s8
+// held as integers X (k_xprep.cuh: X = rne(x' 2^e), |X| < 2^23, three s8
 // digits) and the codes as unsigned bytes: one AND of a code word gives four
 // codes of one "plane" (piece_regs).  The integer tensor cores
-// (mma.m16n8k32.u8.s8, s32 accumulation) form sum_j q_j X_j per digit with
-// no rounding, so the zero point can be taken out exactly:
-//   V = sum_j (q_j - z) X_j = C_l + 256 C_h - z T,   T = sum_j X_j,
+// (mma.m16n8k32.u8.s8, s32 accumulation) form C_d = sum_j q_j d_d(X_j) per
+// digit d with no rounding, so the zero point is taken out exactly:
+//   E_d = C_d - z T_d,   T_d = sum_j d_d(X_j),
+//   V   = E_0 + 256 E_1 + 65536 E_2 = sum_j (q_j - z) X_j,
 // and each block adds s * 2^-e * V to its output row in fp32.  The only
-// roundings are X (for slice elements more than 2^7 below the slice
+// roundings are X (for slice elements more than 2^15 below the slice
 // maximum), the conversion of V to fp32 and the fp32 accumulation -- all
 // relative to sum |x * w_hat|, never to the cancelled sum q*x.
+// 16-bit passthrough blocks (TileQuant abstract) take bf16 mma.m16n8k16 on
+// the block's weights and the slice's bf16 values (a separate build of the
+// kernel, chosen by the layer's MPQ_LAYER_16BIT flag).
 //
 // A block row that lies inside one run is written straight to y.  A block
 // row shared by several runs (the first and last row of a run) is finished
@@ -38,7 +42,8 @@
 // so results are deterministic.
 //
 // Every wait is bounded: after ~2 s it records MPQ_ERR_TIMEOUT and the warp
-// stops computing (its arithmetic is skipped, its bookkeeping still runs).
+// stops computing (its arithmetic is skipped, its bookkeeping still runs);
+// before it leaves it waits, again bounded, for the copies it has in flight.
 #pragma once
 #include "common.cuh"
 #include "k_xprep.cuh"   // XQD_*

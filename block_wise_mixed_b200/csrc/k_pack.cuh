@@ -60,6 +60,11 @@ __device__ __forceinline__ uint32_t f16_bits_small_int(int v) {
     return __half_as_ushort(__int2half_rn(v));  // exact for 0..2048
 }
 
+// STAGED: the source row and the column order are staged in shared memory
+// (about 6 K bytes); rows too long for that (K beyond ~38 K) are read from
+// global memory directly (the row is L1/L2-resident while its groups are
+// quantized).
+template <bool STAGED>
 __global__ void __launch_bounds__(PACK_THREADS)
 k_pack(PackParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -76,9 +81,9 @@ k_pack(PackParams p) {
     const int i_end = min(p.N, i_begin + p.rows_per_cta);
     if (i_begin >= i_end) return;
 
-    if (p.col_perm)
+    if (STAGED && p.col_perm)
         for (int j = tid; j < K; j += PACK_THREADS) cperm[j] = (uint16_t)p.col_perm[j];
-    if (tid == 0) {
+    if (STAGED && tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         fence_mbar_init();
@@ -89,7 +94,12 @@ k_pack(PackParams p) {
         int s = p.row_perm ? p.row_perm[i] : i;
         return p.W + (size_t)s * K;
     };
-    if (tid == 0) {
+    // column c of the reordered row (through col_perm when given)
+    auto col = [&](int c) -> int {
+        if (!p.col_perm) return c;
+        return STAGED ? (int)cperm[c] : __ldg(p.col_perm + c);
+    };
+    if (STAGED && tid == 0) {
         mbar_arrive_expect_tx(&bars[0], row_bytes);
         bulk_g2s(rowbuf0, src_row(i_begin), row_bytes, &bars[0]);
     }
@@ -97,17 +107,19 @@ k_pack(PackParams p) {
     int it = 0;
     for (int i = i_begin; i < i_end; ++i, ++it) {
         const int buf = it & 1;
-        uint16_t* row = buf ? rowbuf1 : rowbuf0;
-        // prefetch the next row into the other buffer (its previous contents
-        // were released by the __syncthreads at the end of the last iteration)
-        if (tid == 0 && i + 1 < i_end) {
-            uint16_t* nrow = buf ? rowbuf0 : rowbuf1;
-            mbar_arrive_expect_tx(&bars[buf ^ 1], row_bytes);
-            bulk_g2s(nrow, src_row(i + 1), row_bytes, &bars[buf ^ 1]);
-        }
-        if (!mbar_wait_bounded(&bars[buf], (uint32_t)((it >> 1) & 1), 2000000000ull)) {
-            if (tid == 0) set_error(p.err, MPQ_ERR_TIMEOUT);
-            return;  // a copy that never lands: stop this CTA
+        const uint16_t* row = STAGED ? (buf ? rowbuf1 : rowbuf0) : src_row(i);
+        if (STAGED) {
+            // prefetch the next row into the other buffer (its previous contents
+            // were released by the __syncthreads at the end of the last iteration)
+            if (tid == 0 && i + 1 < i_end) {
+                uint16_t* nrow = buf ? rowbuf0 : rowbuf1;
+                mbar_arrive_expect_tx(&bars[buf ^ 1], row_bytes);
+                bulk_g2s(nrow, src_row(i + 1), row_bytes, &bars[buf ^ 1]);
+            }
+            if (!mbar_wait_bounded(&bars[buf], (uint32_t)((it >> 1) & 1), 2000000000ull)) {
+                if (tid == 0) set_error(p.err, MPQ_ERR_TIMEOUT);
+                return;  // a copy that never lands: stop this CTA
+            }
         }
 
         const int nb = i >> 6, r = i & 63;
@@ -124,8 +136,7 @@ k_pack(PackParams p) {
                 bool finite = true, in_range = true;
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    const int c = p.col_perm ? (int)cperm[c0 + e4] : c0 + e4;
-                    wb[e4] = row[c];
+                    wb[e4] = row[col(c0 + e4)];
                     const float v = __uint_as_float(((uint32_t)wb[e4]) << 16);
                     finite &= isfinite(v);
                     in_range &= fabsf(v) <= 65504.f;
@@ -151,8 +162,7 @@ k_pack(PackParams p) {
             const int c0 = kb * 128 + 4 * lane;
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
-                int c = p.col_perm ? (int)cperm[c0 + e4] : c0 + e4;
-                w[e4] = __uint_as_float(((uint32_t)row[c]) << 16);
+                w[e4] = __uint_as_float(((uint32_t)row[col(c0 + e4)]) << 16);
             }
             bool finite = true;
             float lo = 0.f, hi = 0.f;

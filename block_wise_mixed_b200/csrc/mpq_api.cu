@@ -33,6 +33,7 @@ constexpr int kMaxDecodeTokens = DEC_MAX_TOKENS;   // tokens per decode launch
 // 28672 x 8192 layers).
 constexpr int kDecodeMaxM = 8;
 constexpr int kPackRowsPerCta = 1;
+constexpr size_t kPackStagedMaxSmem = 227 * 1024;   // the sm_100 maximum per CTA
 
 inline size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -311,6 +312,7 @@ std::atomic<uint64_t> g_decode_attr_g{0};
 std::atomic<uint64_t> g_prefill_attr{0};
 std::atomic<uint64_t> g_prefill_attr256{0};
 std::atomic<uint64_t> g_unperm_attr{0};
+std::atomic<uint64_t> g_pack_attr{0};
 
 // cuTensorMapEncodeTiled from the driver, looked up through the runtime.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -436,12 +438,18 @@ mpq_status mpq_pack_timed(const mpq_layout* L, const void* W_dev, const uint8_t*
     p.K = L->K;
     p.KB = L->KB;
     p.rows_per_cta = kPackRowsPerCta;
+    // two row buffers, the column order as uint16, two mbarriers; rows longer
+    // than that allows are read from global memory by the unstaged kernel
     const size_t row_bytes = (size_t)L->K * 2;
     const size_t smem = 2 * row_bytes + ((row_bytes + 15) & ~size_t(15)) + 64;
-    e = cudaFuncSetAttribute(k_pack, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    const bool staged = smem <= kPackStagedMaxSmem;
+    if (staged) {
+        e = ensure_smem_attr(k_pack<true>, (int)kPackStagedMaxSmem, g_pack_attr);
+        if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    }
     const int grid = (L->N + kPackRowsPerCta - 1) / kPackRowsPerCta;
-    k_pack<<<grid, PACK_THREADS, smem, s>>>(p);
+    if (staged) k_pack<true><<<grid, PACK_THREADS, smem, s>>>(p);
+    else k_pack<false><<<grid, PACK_THREADS, 0, s>>>(p);
     e = cudaGetLastError();
     if (e == cudaSuccess && ev_end) e = cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s);
     return cuda_status(e);

@@ -473,3 +473,18 @@ def test_sixteen_bit_block_without_flag(mpq, oracle, M):
     R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
     y_ref, bnd = oracle.linear(R, synth.make_x(9401 + M, M, L.K))
     assert_y_close(run_linear(mpq, P, synth.make_x(9401 + M, M, L.K)), y_ref, bnd)
+
+
+@pytest.mark.parametrize("K", [40960, 65536])
+def test_pack_long_rows(mpq, oracle, K):
+    """Rows too long to stage in shared memory (6 K bytes > 227 KB): the pack
+    reads them from global memory; byte-exact against the oracle, and the
+    layer matches the oracle on the decode and tensor-core paths."""
+    L = synth.make_layer("long", 128, K, 2.5, 9500 + K // 4096, "random")
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    assert_pack_equal(P, R)
+    for M in (1, 40):
+        x = synth.make_x(9600 + M, M, K)
+        y_ref, bnd = oracle.linear(R, x)
+        assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
