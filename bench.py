@@ -2,15 +2,16 @@
 """Benchmark of the block-wise mixed-precision weight-only linear layer.
 
 Headline step: one Llama-3-70B decoder layer at M=1 (one decode token) --
-the seven mpq_linear calls q, k, v, o, gate, up, down (8192 hidden, 28672
-MLP, 2.1 average bits, channel orders on all but q and k), each an
-activation reorder + mixed-precision GEMV + inverse output reorder.  The
+its seven projections q, k, v, o, gate, up, down (8192 hidden, 28672 MLP,
+2.1 average bits, channel orders on all but q and k), each an activation
+reorder + mixed-precision GEMV + inverse output reorder; k and v, which
+share x, go through one mpq_linear_group call (one launch).  The
 steps cycle through replicas of the packed layer whose total size is more
 than 4x the L2 cache, and L2 is flushed (a buffer of twice its size is
 written) right before the timed replay, so every timed step streams its
 weights from HBM whatever the step count.
 
-value = algorithmic HBM bytes of the seven calls / device time of a step
+value = algorithmic HBM bytes of the seven projections / device time of a step
 (GB/s, summed over ranks, time = max over ranks).  The same line carries the
 tensor-core path on the Llama-3-8B layer at M = 512 and 2048 (TFLOP/s), the
 full-layer mpq_pack time and the 4096x4096 (Llama-2-7B attention) layer at
@@ -241,11 +242,33 @@ def packed_bytes(P):
     return lay.codes_bytes + 4 * lay.n_sz + 16 * lay.NB * lay.KB + 4 * (lay.N + lay.K)
 
 
-class Workload:
-    """A step of one mpq_linear call per layer at M tokens, over replicas of
-    the packed layers whose total size is at least 4x L2."""
+# The decoder layer's calls: q, then k and v as one mpq_linear_group call
+# (they share x; at M=1 both take the one-token path, so the group is one
+# launch), o, gate, up, down.  x sources as in the model: q, k, v read the
+# normed hidden state, o the attention output, gate and up the normed hidden
+# state of the MLP, down the MLP activation.
+DECODER_GROUPS = [[0], [1, 2], [3], [4], [5], [6]]
+DECODER_X_SRC = [0, 0, 0, 1, 2, 2, 3]
 
-    def __init__(self, mpq, layers, M, device, seed=99, max_replicas=64):
+
+def headline_desc(layers):
+    """The headline workload, as both arms name it in `config`."""
+    avg_bits = float(np.mean(np.concatenate([L.bits for L in layers])))
+    f0 = float(np.mean(np.concatenate([L.bits == 0 for L in layers])))
+    return ("Llama-3-70B decoder layer at M=1: q 8192x8192, k,v 1024x8192, "
+            "o 8192x8192, gate,up 28672x8192, down 8192x28672 (856 M weights), "
+            "avg %.2f bits (f0=%.3f), saliency channel orders (identity for q,k); "
+            "one step = q, k+v (one mpq_linear_group call), o, gate, up, down; "
+            "q, k, v share x, gate and up share x" % (avg_bits, f0))
+
+
+class Workload:
+    """A step of mpq_linear calls at M tokens -- one per layer, or one
+    mpq_linear_group call per entry of `groups` -- over replicas of the
+    packed layers whose total size is at least 4x L2.  x_src[i] names the
+    activation that layer i reads (layers with the same source share it)."""
+
+    def __init__(self, mpq, layers, M, device, seed=99, max_replicas=64, groups=None, x_src=None):
         import torch
         from block_wise_mixed_b200 import synth
         self.mpq, self.layers, self.M, self.device = mpq, layers, M, device
@@ -258,11 +281,21 @@ class Workload:
         per_step = sum(packed_bytes(P) for P in self.packs)
         self.R = int(max(2, min(max_replicas, np.ceil(4 * self.l2 / max(per_step, 1)))))
         self.reps = [self.packs] + [[clone_layer(P) for P in self.packs] for _ in range(self.R - 1)]
-        self.x_bits = [synth.make_x(synth.seed_of(seed, i), M, L.K) for i, L in enumerate(layers)]
-        self.x = [torch.from_numpy(xb.view(np.int16)).to(device) for xb in self.x_bits]
+        self.groups = groups if groups is not None else [[i] for i in range(len(layers))]
+        x_src = x_src if x_src is not None else list(range(len(layers)))
+        srcs = {}
+        for i, L in enumerate(layers):
+            if x_src[i] not in srcs:
+                srcs[x_src[i]] = synth.make_x(synth.seed_of(seed, x_src[i]), M, L.K)
+        self.x_bits = [srcs[x_src[i]] for i in range(len(layers))]
+        xdev = {k: torch.from_numpy(v.view(np.int16)).to(device) for k, v in srcs.items()}
+        self.x = [xdev[x_src[i]] for i in range(len(layers))]
         self.y = [torch.empty((M, L.N), dtype=torch.float32, device=device) for L in layers]
         self.ws = torch.zeros(max(mpq.linear_workspace_size(P, M) for P in self.packs),
                               dtype=torch.uint8, device=device)
+        self.gws = {tuple(g): torch.zeros(mpq.linear_group_workspace_size([self.packs[i] for i in g], M),
+                                          dtype=torch.uint8, device=device)
+                    for g in self.groups if len(g) > 1}
         self.flush = torch.empty(2 * self.l2, dtype=torch.uint8, device=device)
         torch.cuda.synchronize(device)
         lays = [P.layout for P in self.packs]
@@ -273,13 +306,23 @@ class Workload:
                                        L.row_perm is not None) for L, l in zip(layers, lays))
         self.flops = sum(2.0 * M * L.N * L.K * (1.0 - float((L.bits == 0).mean())) for L in layers)
         self.dense_flops = sum(2.0 * M * L.N * L.K for L in layers)
-        self.launches = sum(launches_per_call(l, M, L.row_perm is not None)
-                            for L, l in zip(layers, lays))
+        self.launches = 0
+        for g in self.groups:
+            per = [launches_per_call(lays[i], M, layers[i].row_perm is not None) for i in g]
+            one_launch = len(g) > 1 and M == 1 and all(
+                lays[i].NB * lays[i].KB <= 2 * lays[i].n_units for i in g)
+            self.launches += 1 if one_launch else sum(per)
         self.footprint = self.R * per_step
 
     def step(self, r):
-        for P, x, y in zip(self.reps[r % self.R], self.x, self.y):
-            self.mpq.linear(P, x, y, self.ws)
+        rep = self.reps[r % self.R]
+        for g in self.groups:
+            if len(g) == 1:
+                i = g[0]
+                self.mpq.linear(rep[i], self.x[i], self.y[i], self.ws)
+            else:
+                self.mpq.linear_group([rep[i] for i in g], self.x[g[0]], [self.y[i] for i in g],
+                                      self.gws[tuple(g)])
 
     def flush_l2(self):
         self.flush.fill_(1)
@@ -516,7 +559,7 @@ def run_gpu(args):
     if args.layer_quick:
         # the headline step's timed loop only (for the launch list)
         layers = [synth.config_layer(HEADLINE_CFG, p) for p in range(7)]
-        wl = Workload(mpq, layers, HEADLINE_M, device)
+        wl = Workload(mpq, layers, HEADLINE_M, device, groups=DECODER_GROUPS, x_src=DECODER_X_SRC)
         ms, _ = wl.time_steps(args.steps, args.warmup, world, soak_s=0.0)
         if rank == 0:
             print(json.dumps({"layer_quick": True, "us_per_step": ms * 1e3,
@@ -524,7 +567,7 @@ def run_gpu(args):
         return
 
     layers = [synth.config_layer(HEADLINE_CFG, p) for p in range(7)]
-    wl = Workload(mpq, layers, HEADLINE_M, device)
+    wl = Workload(mpq, layers, HEADLINE_M, device, groups=DECODER_GROUPS, x_src=DECODER_X_SRC)
     sampler = ClockSampler(local)
     ms_step, clocks = wl.time_steps(args.steps, args.warmup, world, sampler=sampler)
     k_ms, k_per = wl.time_kernels(args.steps)
@@ -538,17 +581,12 @@ def run_gpu(args):
     # time is the conservative denominator and can never exceed the step
     achieved = wl.kbytes / (ms_step * 1e-3) / 1e9
     traffic = load_traffic("k_decode", "llama70b_layer_m1")
-    avg_bits = float(np.mean(np.concatenate([L.bits for L in layers])))
-    f0 = float(np.mean(np.concatenate([L.bits == 0 for L in layers])))
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp16", "data": "synthetic",
-        "config": {"workload": "Llama-3-70B decoder layer at M=1: q 8192x8192, k,v 1024x8192, "
-                               "o 8192x8192, gate,up 28672x8192, down 8192x28672 (856 M weights), "
-                               "avg %.2f bits (f0=%.3f), saliency channel orders (identity for q,k); "
-                               "one step = 7 mpq_linear calls" % (avg_bits, f0),
+        "dtype": "int8", "data": "synthetic",
+        "config": {"workload": headline_desc(layers),
                    "M": HEADLINE_M, "layer_bytes": int(wl.bytes), "replicas": wl.R,
                    "l2": "inputs larger than L2: %d replicas of the packed layer cycled (%.0f MB, "
                          "L2 %.0f MB), L2 flushed before the timed replay"
@@ -557,7 +595,7 @@ def run_gpu(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                     "kernel": "k_decode (the 7 decode launches of a step)",
+                     "kernel": "k_decode, k_decode_group (the 6 decode launches of a step)",
                      "peak_source": peak_src,
                      "kernel_us_per_step": round(ms_step * 1e3, 2),
                      "kernel_bytes_per_step": int(wl.kbytes),
@@ -636,7 +674,12 @@ def run_reference(args):
     from block_wise_mixed_b200 import synth
     cfg = HEADLINE_CFG if args.cfg is None else args.cfg     # --cfg: another workload's layers
     layers = [synth.config_layer(cfg, p) for p in range(len(synth.CONFIGS[cfg]["layers"]))]
-    xs = [synth.make_x(synth.seed_of(99, i), HEADLINE_M, L.K) for i, L in enumerate(layers)]
+    if cfg == HEADLINE_CFG:   # the same activations as the GPU arm's step
+        src = {j: synth.make_x(synth.seed_of(99, j), HEADLINE_M, layers[DECODER_X_SRC.index(j)].K)
+               for j in sorted(set(DECODER_X_SRC))}
+        xs = [src[DECODER_X_SRC[i]] for i in range(len(layers))]
+    else:
+        xs = [synth.make_x(synth.seed_of(99, i), HEADLINE_M, L.K) for i, L in enumerate(layers)]
     packs = oracle_packs(layers)
     stride = 64      # each step: 1/64 of the output rows of every projection
     for _ in range(max(args.warmup, 3)):
@@ -654,8 +697,10 @@ def run_reference(args):
            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": "%s at M=1, fp64 CPU oracle on 1/%d of the output rows"
-                                  % (synth.CONFIGS[cfg]["desc"], stride), "M": HEADLINE_M},
+           "config": {"workload": (headline_desc(layers) if cfg == HEADLINE_CFG else
+                                   "%s at M=1" % synth.CONFIGS[cfg]["desc"]),
+                      "M": HEADLINE_M,
+                      "oracle_sample": "fp64 CPU oracle on 1/%d of the output rows" % stride},
            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": cores,
                             "kind": "oracle", "sample": sample},
            "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
