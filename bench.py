@@ -68,10 +68,11 @@ def kernel_bytes(N, K, M, codes_bytes, n_sz, T, has_rp):
     return codes_bytes + 4 * n_sz + 16 * T + 4 * (N if has_rp else 0) + 2 * M * K + 4 * M * N
 
 
-def source_hash():
+def source_hash(names=None):
+    """Hash of the kernel sources (all of csrc/, or the listed files)."""
     h = hashlib.sha1()
     d = os.path.join(ROOT, "block_wise_mixed_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    for name in sorted(names if names else os.listdir(d)):
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -87,7 +88,7 @@ def load_traffic(kernel: str, workload: str):
     except (OSError, ValueError):
         return None
     e = d.get(kernel, {}).get(workload)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(e.get("sources")):
         return None
     return e.get("dram_bytes_per_step", e.get("dram_bytes_per_launch"))
 

@@ -16,6 +16,7 @@
 #include "k_decode.cuh"
 #include "k_pack.cuh"
 #include "k_prefill.cuh"
+#include "k_tcdec.cuh"
 #include "k_xprep.cuh"
 #include "k_ycast.cuh"
 
@@ -32,6 +33,13 @@ constexpr int kMaxDecodeTokens = DEC_MAX_TOKENS;   // tokens per decode launch
 // call at M = 8 and twice as much at M = 16 (measured on the 14336 x 4096 and
 // 28672 x 8192 layers).
 constexpr int kDecodeMaxM = 8;
+// 9..16 tokens on layers of at least 100 tiles of 128 rows: the integer
+// tensor-core kernel (k_tcdec; one CTA per tile, all k blocks); smaller
+// layers, and layers with 16-bit blocks, take k_prefill, which splits k
+// across CTAs (measured: the 8192-row q projection at 16 tokens 68 us with
+// 64 k_tcdec CTAs against 38 us split)
+constexpr int kTcDecMaxM = 16;
+constexpr int kTcDecMinTiles = 100;
 constexpr int kPackRowsPerCta = 1;
 constexpr size_t kPackStagedMaxSmem = 227 * 1024;   // the sm_100 maximum per CTA
 
@@ -542,11 +550,84 @@ DecodeParams decode_params(const mpq_layer* layer, const void* x_dev, int32_t M,
     return dp;
 }
 
+std::atomic<uint64_t> g_tcdec_attr1{0};
+std::atomic<uint64_t> g_tcdec_attr2{0};
+
+template <int WPQ>
+size_t tcdec_smem_bytes(int KB) {
+    return sizeof(TcSmem<TC_MP, WPQ>) + 1024 + (size_t)2 * KB;
+}
+
+template <int WPQ>
+mpq_status tcdec_launch(const TcParams& tp, int tiles, cudaStream_t s, cudaLaunchAttribute* pdl,
+                        std::atomic<uint64_t>& attr) {
+    const size_t smem = tcdec_smem_bytes<WPQ>(tp.KB);
+    const size_t cap = WPQ == 2 ? 113 * 1024 : 227 * 1024;   // two CTAs per SM, or one
+    if (smem > cap) return MPQ_ERR_SHAPE;
+    cudaError_t e = ensure_smem_attr(k_tcdec<TC_MP, WPQ>, (int)cap, attr);
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    cudaLaunchConfig_t c{};
+    c.gridDim = dim3((unsigned)tiles);
+    c.blockDim = dim3(TcCfg<TC_MP, WPQ>::THREADS);
+    c.dynamicSmemBytes = smem;
+    c.stream = s;
+    c.attrs = pdl;
+    c.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&c, k_tcdec<TC_MP, WPQ>, tp));
+}
+
+// 9..16 tokens on a layer without 16-bit blocks: activation records
+// (k_xprep_tcdec), then the integer tensor-core kernel, chained by
+// programmatic dependent launch.  Grids of at most one wave take the
+// variant with one CTA per SM and more worker warps; larger grids the
+// one with two CTAs per SM (one wave instead of two).
+mpq_status tcdec_run(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev, const LinearWs& w,
+                     cudaStream_t s, cudaLaunchConfig_t xc, void* ev_begin, void* ev_end) {
+    const int KB = layer->K / 128, NB = layer->N / 64;
+    const int tiles = (NB + 1) / 2;
+    XprepTcParams xt{};
+    xt.x = static_cast<const uint16_t*>(x_dev);
+    xt.col_perm = layer->col_perm;
+    xt.rec = reinterpret_cast<uint8_t*>(w.xq);
+    xt.M = M;
+    xt.K = layer->K;
+    xt.MP = TC_MP;
+    xt.NP = 3 * TC_MP;
+    xt.REC = TcCfg<TC_MP, 2>::REC;
+    const int items = KB * TC_MP, per = XPREP_THREADS / 32;
+    xc.gridDim = dim3((unsigned)((items + per - 1) / per));
+    cudaError_t e = cudaLaunchKernelEx(&xc, k_xprep_tcdec, xt);
+    if (e != cudaSuccess) return MPQ_ERR_CUDA;
+    TcParams tp{};
+    tp.codes = static_cast<const uint8_t*>(layer->codes);
+    tp.table = layer->table;
+    tp.scales = layer->scales;
+    tp.zeros = layer->zeros;
+    tp.row_perm = layer->row_perm;
+    tp.rec = xt.rec;
+    tp.y = y_dev;
+    tp.err = w.err;
+    tp.N = layer->N;
+    tp.K = layer->K;
+    tp.NB = NB;
+    tp.KB = KB;
+    tp.M = M;
+    if (ev_begin && cudaEventRecord(static_cast<cudaEvent_t>(ev_begin), s) != cudaSuccess) return MPQ_ERR_CUDA;
+    cudaLaunchAttribute* pdl = const_cast<cudaLaunchAttribute*>(xc.attrs);
+    const mpq_status st = tiles <= 148 ? tcdec_launch<4>(tp, tiles, s, pdl, g_tcdec_attr1)
+                                       : tcdec_launch<2>(tp, tiles, s, pdl, g_tcdec_attr2);
+    if (st != MPQ_OK) return st;
+    if (ev_end && cudaEventRecord(static_cast<cudaEvent_t>(ev_end), s) != cudaSuccess) return MPQ_ERR_CUDA;
+    return MPQ_OK;
+}
+
 // mpq_linear on a carved workspace (arguments already checked).
 mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, float* y_dev,
                       const LinearWs& w, cudaStream_t s, void* ev_begin, void* ev_end) {
     const int NB = layer->N / 64, KB = layer->K / 128;
     const bool use_tc = M > kDecodeMaxM;
+    const bool use_tcdec = use_tc && M <= kTcDecMaxM && (layer->flags & MPQ_LAYER_16BIT) == 0 &&
+                           (NB + 1) / 2 >= kTcDecMinTiles;
     if (!use_tc && (uint64_t)KB * (uint64_t)M * XQD_REC >= (1ull << 32)) return MPQ_ERR_SHAPE;
     const bool fused = !use_tc && fused_one_token(layer, M);
     XprepParams xp{};
@@ -570,6 +651,8 @@ mpq_status linear_run(const mpq_layer* layer, const void* x_dev, int32_t M, floa
     xc.attrs = pdl;
     xc.numAttrs = 1;
     cudaError_t e;
+    if (use_tcdec)
+        return tcdec_run(layer, x_dev, M, y_dev, w, s, xc, ev_begin, ev_end);
     if (use_tc) {
         xp.counters = nullptr;
         // few tokens: several CTAs per token, about two waves in all

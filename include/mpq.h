@@ -212,12 +212,14 @@ size_t mpq_linear_workspace_size(const mpq_layer* layer, int32_t M);
  *           cudaMemset); every call that ends without a device error leaves
  *           the parts that must start at zero at zero, so it can be reused
  *           as is (zero it again after a device error).
- * Uses a memory-bound decode kernel (integer tensor cores) for M <= 8 and a
- * tcgen05 tensor-core kernel for larger M.  Non-finite x gives non-finite y
+ * Uses a memory-bound decode kernel (integer tensor cores) for M <= 8; for
+ * 9 <= M <= 16 on layers of at least 100 tiles of 128 rows without 16-bit
+ * blocks, the same integer arithmetic on tcgen05 (kind::i8); otherwise a
+ * tcgen05 kernel on dequantized fp16 tiles.  Non-finite x gives non-finite y
  * (no error).  Activations are scaled by exact powers of two (per 128-column
- * slice into 23-bit integers for M <= 8, per token into fp16 above); a
- * slice element more than 2^15 below the slice maximum is rounded to 2^-23
- * of that maximum.
+ * slice into 23-bit integers on the integer paths, per token into fp16 on
+ * the fp16 path); a slice element more than 2^15 below the slice maximum is
+ * rounded to 2^-23 of that maximum.
  * Host errors: ARG, SHAPE, WORKSPACE; device (mpq_check): TIMEOUT, BITS (a
  * 16-bit block in a layer whose flags lack MPQ_LAYER_16BIT). */
 mpq_status mpq_linear(const mpq_layer* layer, const void* x_dev, int32_t M,

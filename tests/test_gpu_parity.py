@@ -488,3 +488,16 @@ def test_pack_long_rows(mpq, oracle, K):
         x = synth.make_x(9600 + M, M, K)
         y_ref, bnd = oracle.linear(R, x)
         assert_y_close(run_linear(mpq, P, x), y_ref, bnd)
+
+
+@pytest.mark.parametrize("M", [9, 13, 16])
+def test_integer_tensor_core_mid_batch(mpq, oracle, M):
+    """9..16 tokens on a layer of >= 100 row tiles: the integer tensor-core
+    kernel.  An odd number of block rows (the last tile half empty), every
+    width incl. 0-bit blocks, random orders; element by element."""
+    L = synth.make_layer("itc", 64 * 201, 1024, 3.0, 9700 + M, "random")
+    P = pack_gpu(mpq, L)
+    R = oracle.pack(L.W, L.bits, L.row_perm, L.col_perm)
+    x = synth.make_x(9800 + M, M, L.K)
+    y_ref, bnd = oracle.linear(R, x)
+    assert_y_close(run_linear(mpq, P, x), y_ref, bnd)

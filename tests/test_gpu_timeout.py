@@ -35,11 +35,13 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("M", [1, 3, 40])     # fused one-token decode, decode + prologue, tensor core
-def test_linear_wait_runs_out(libs, oracle, M):
+# fused one-token decode, decode + prologue, fp16 tensor core, and the
+# integer tensor-core kernel (9..16 tokens on a layer of >= 100 row tiles)
+@pytest.mark.parametrize("M,shape", [(1, None), (3, None), (40, None), (12, (64 * 201, 1024))])
+def test_linear_wait_runs_out(libs, oracle, M, shape):
     import torch
     mpq, _lib, wt = libs
-    L = synth.config_layer(1, 0)
+    L = synth.config_layer(1, 0) if shape is None else synth.make_layer("wt", shape[0], shape[1], 3.0, 77, "random")
     P = mpq.pack(torch.from_numpy(L.W.view(np.int16)).cuda(), L.bits, L.row_perm, L.col_perm)
     x = torch.from_numpy(synth.make_x(11, M, L.K).view(np.int16)).cuda()
     y = torch.empty((M, L.N), dtype=torch.float32, device="cuda")

@@ -39,11 +39,13 @@ def _layer(spec):
     return synth.make_layer("tc", N, K, 3.0, 4000 + N + K, "random")
 
 
-# Decode kernel (M <= 16) and tensor-core kernel (M > 16): the latter carves
-# its split-K partial sums out of the static array (N=512, K=128*11 at M=40
-# splits the k blocks in two) and reorders rows with a second kernel.
+# Decode kernel (M <= 8), integer tensor-core kernel (9..16, its activation
+# records in the static array) and the fp16 tensor-core kernel (M > 16): the
+# latter carves its split-K partial sums out of the static array (N=512,
+# K=128*11 at M=40 splits the k blocks in two) and reorders rows with a
+# second kernel.
 @pytest.mark.parametrize("spec,M", [(("cfg", 1), 1), (("cfg", 1), 5), (("cfg", 2), 1),
-                                    (("cfg", 2), 8), (("cfg", 1), 33),
+                                    (("cfg", 2), 8), (("tc", 64 * 201, 1024), 12), (("cfg", 1), 33),
                                     (("tc", 512, 128 * 11), 40)])
 def test_noalloc_matches_workspace_entry_point(mpq, oracle, spec, M):
     import torch
