@@ -93,16 +93,20 @@ def load_traffic(kernel: str, workload: str):
     return e.get("dram_bytes_per_step", e.get("dram_bytes_per_launch"))
 
 
-def launches_per_call(lay, M, has_row_perm):
+def launches_per_call(lay, M, has_row_perm, has_16bit=False):
     """Kernels one mpq_linear call launches (the library's dispatch rule):
     M <= 8 -- the activation prologue unless M == 1 on a layer whose runs
     hold at most two blocks on average (the decode kernel then builds its own
-    activation records), plus one decode launch; M > 8 -- the prologue, the
+    activation records), plus one decode launch; 9..16 tokens on a layer of
+    at least 100 tiles of 128 rows without 16-bit blocks -- the record
+    prologue and the integer tensor-core kernel; otherwise the prologue, the
     tensor-core kernel and, when the rows are reordered (or k is split), the
     reordering kernel."""
     if M <= 8:
         fused = M == 1 and lay.NB * lay.KB <= 2 * lay.n_units
         return (0 if fused else 1) + (M + 7) // 8
+    if M <= 16 and (lay.NB + 1) // 2 >= 100 and not has_16bit:
+        return 2
     return 2 + (1 if has_row_perm else 0)
 
 
@@ -309,7 +313,8 @@ class Workload:
         self.dense_flops = sum(2.0 * M * L.N * L.K for L in layers)
         self.launches = 0
         for g in self.groups:
-            per = [launches_per_call(lays[i], M, layers[i].row_perm is not None) for i in g]
+            per = [launches_per_call(lays[i], M, layers[i].row_perm is not None,
+                                     bool((layers[i].bits == 16).any())) for i in g]
             one_launch = len(g) > 1 and M == 1 and all(
                 lays[i].NB * lays[i].KB <= 2 * lays[i].n_units for i in g)
             self.launches += 1 if one_launch else sum(per)
