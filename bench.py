@@ -493,6 +493,31 @@ def run_tensor_core(mpq, layers, device, peaks, steps):
     return out
 
 
+def run_mid_batch(mpq, device, peaks, steps):
+    """Mid-size batches on the 8B MLP gate (14336x4096, 3.0 bits) and the
+    70B gate (28672x8192, 2.1 bits) at 16 tokens (the integer tensor-core
+    kernel) and 32 (the fp16 one): HBM GB/s of one call, replicas cycled,
+    L2 flushed before the timed replay.  A failure is reported in the line
+    instead of ending the run."""
+    from block_wise_mixed_b200 import synth
+    out = {}
+    for cfg, proj, name in ((3, 0, "llama3_8b_gate"), (4, 4, "llama3_70b_gate")):
+        try:
+            L = synth.config_layer(cfg, proj)
+            for M in (16, 32):
+                wl = Workload(mpq, [L], M, device)
+                ms, _ = wl.time_steps(steps, 3, 1, soak_s=0.0)
+                gbs = wl.bytes / (ms * 1e-3) / 1e9
+                out["%s_M%d" % (name, M)] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1),
+                                             "frac": round(gbs / peaks["hbm_gbs"], 4), "replicas": wl.R}
+                wl.release()
+                del wl
+            del L
+        except Exception as ex:   # keep the rest of the line
+            out[name] = {"error": repr(ex)[:200]}
+    return out
+
+
 def run_allocation(mpq, device, peaks):
     """Budgeted bit allocation (mpq_allocate_bits) over the block count of the
     Llama-3-70B decoder layer: device time with CUDA events, search
@@ -640,6 +665,7 @@ def run_gpu(args):
                                          "frac": round(attn.bytes / (ms * 1e-3) / 1e9 /
                                                        peaks["hbm_gbs"], 4)}
         attn.release()
+        res["mid_batch"] = run_mid_batch(mpq, device, peaks, max(min(args.steps, 50), 16))
     if args.extra and rank == 0:
         res["extra"] = run_extra(mpq, args, device, peaks)
     if world > 1:
