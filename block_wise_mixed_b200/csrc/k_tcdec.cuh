@@ -26,10 +26,10 @@
 // the warps in between expand and accumulate.  Measured on B200: faster
 // than the dequantizing fp16 kernel up to 16 tokens (the 70B gate
 // projection at 16 tokens 99 vs 130 us), slower above, where k_prefill
-// stays in use.  16-bit passthrough blocks are
-// not handled here (layers flagged MPQ_LAYER_16BIT take k_prefill).  All
-// waits are bounded (MPQ_ERR_TIMEOUT), with a bounded drain of copies and
-// MMAs in flight before TMEM is freed.
+// stays in use.  16-bit passthrough blocks are not handled here (layers
+// flagged MPQ_LAYER_16BIT take k_prefill).  All waits are bounded
+// (MPQ_ERR_TIMEOUT), with a bounded drain of copies and MMAs in flight
+// before TMEM is freed.
 #pragma once
 #include <cuda.h>
 
